@@ -1,0 +1,349 @@
+"""Benchmark: MXFP4 MoE expert block, forward + input-gradient backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = mxfp4_moe_forward + mxfp4_moe_backward_input over one batch of T synthetic tokens
+(seeded; inputs resident in HBM).  With N > 1 (launched by torch.distributed.run) every rank
+runs its own independent batch (the layer has no weight gradient and every token is
+independent, so data parallelism needs no collective); the timing is the max over ranks and
+`value` counts all ranks' tokens.  Prints one JSON line on rank 0.
+
+`--impl reference` times the fp64 CPU oracle instead (rank 0 only), on a bounded token sample
+of each step's workload, on this host's cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd+bwd(dX) tokens/s, 1×B200, gpt-oss-20b shape; % tensor roofline"
+DEFAULT_WORKLOAD = "gpt-oss-20b-moe-T8192"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--kernel-table", action="store_true", help="print the per-kernel table to stderr")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads") or 0) for i in threadpool_info()) or os.cpu_count()
+    except Exception:  # pragma: no cover
+        n = os.cpu_count()
+    return int(n)
+
+
+def oracle_sample(wl, seed, n_tokens, inp=None):
+    """Time the oracle (forward + backward) on the first n_tokens of the workload's batch."""
+    from mxfp4_quantized_moe_b200 import inputs
+    from oracle import mxfp4_oracle as O
+    if inp is None:
+        inp = inputs.make_workload(wl, seed)
+    sel = np.arange(min(n_tokens, wl.T))
+    n = inputs.as_numpy(inp, sel)
+    t0 = time.perf_counter()
+    f = O.moe_forward(n["x"], n["logits"], n["W"], wl.k)
+    O.moe_backward(n["dy"], f, n["W"])
+    dt = time.perf_counter() - t0
+    return len(sel), dt
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def run_reference(args, rank):
+    from mxfp4_quantized_moe_b200 import inputs
+    if rank != 0:
+        return
+    wl = inputs.WORKLOADS[args.workload]
+    inp = inputs.make_workload(wl, args.seed)
+    # the oracle dequantizes every expert a sample touches (about 1-2 s per expert in fp64), so
+    # each step samples one token: its k experts; the whole run stays within a few minutes
+    n_tok = 1
+    for _ in range(args.warmup):
+        oracle_sample(wl, args.seed, n_tok, inp)
+    times = []
+    for _ in range(args.steps):
+        n, dt = oracle_sample(wl, args.seed, n_tok, inp)
+        times.append(dt)
+    tot = sum(times)
+    value = n_tok * args.steps / tot
+    cores = cpu_threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                   "sample_tokens_per_step": n_tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_tok} tokens of the {wl.name} batch per step (fwd+bwd)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import torch
+    import torch.distributed as dist
+    from mxfp4_quantized_moe_b200 import inputs, moe
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    wl = inputs.WORKLOADS[args.workload]
+    if wl.layers != 1:
+        raise SystemExit("bench times single-layer workloads")
+    # each rank draws its own batch (seed + rank); the weights are the same on every rank
+    inp = inputs.make_workload(wl, args.seed)
+    if rank:
+        xr = inputs.make_workload(wl, args.seed + 1000 * rank)
+        inp = dict(inp, x=xr["x"], logits=xr["logits"], dy=xr["dy"])
+    shape = moe.MoeShape(wl.T, wl.H, wl.I, wl.E, wl.k)
+    w = moe.weights_to(inp, dev)
+    x = inp["x"].to(dev)
+    lg = inp["logits"].to(dev)
+    dy = inp["dy"].to(dev)
+    ws = moe.alloc_workspace(shape, dev)
+    wt = moe.transpose_weights(shape, w)
+    y = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+    dx = torch.empty_like(y)
+    dtw = torch.empty(wl.T, wl.k, dtype=torch.float32, device=dev)
+    dl = torch.empty(wl.T, wl.E, dtype=torch.float32, device=dev)
+
+    def step():
+        moe.forward(shape, w, x, lg, ws, y=y)
+        moe.backward_input(shape, w, wt, dy, ws, dx=dx, d_topk_w=dtw, d_logits=dl)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc, where = moe.device_check(ws)
+    if rc != 0:
+        raise SystemExit(f"device error {rc} at {where:#x}")
+
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    moe.profile_begin()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    kt = moe.profile_end()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    clk = clocks.stop() if rank == 0 else None
+    rc, where = moe.device_check(ws)
+    if rc != 0:
+        raise SystemExit(f"device error {rc} at {where:#x}")
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end through the public API with host buffers ----------------------------
+    hx = inp["x"].pin_memory()
+    hlg = inp["logits"].pin_memory()
+    hdy = inp["dy"].pin_memory()
+    hy = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+    hdx = torch.empty_like(hy).pin_memory()
+    hdtw = torch.empty(wl.T, wl.k, dtype=torch.float32).pin_memory()
+    hdl = torch.empty(wl.T, wl.E, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        x.copy_(hx, non_blocking=True)
+        lg.copy_(hlg, non_blocking=True)
+        dy.copy_(hdy, non_blocking=True)
+        step()
+        hy.copy_(y, non_blocking=True)
+        hdx.copy_(dx, non_blocking=True)
+        hdtw.copy_(dtw, non_blocking=True)
+        hdl.copy_(dl, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t2 = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t2.item())
+    h2d = sum(int(v.numel() * v.element_size()) for v in (hx, hlg, hdy))
+    d2h = sum(int(v.numel() * v.element_size()) for v in (hy, hdx, hdtw, hdl))
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    T, H, I, E, k = wl.T, wl.H, wl.I, wl.E, wl.k
+    A = T * k
+    flop_step = 12.0 * A * H * I
+    value = T * world * args.steps / (ms_max / 1e3)
+    pk = peaks()
+    # dominant kernel: largest summed device time inside the timed region
+    gemm_flops = {"gemm_gate_up_glu": 2.0 * A * H * 2 * I, "gemm_down_scatter": 2.0 * A * I * H,
+                  "gemm_dact_glu_bwd": 2.0 * A * H * I, "gemm_dx_scatter": 2.0 * A * 2 * I * H}
+    top = max(kt.items(), key=lambda kv: kv[1][1])
+    name, (launches, tot) = top
+    roof = None
+    if name in gemm_flops:
+        avg_ms = tot / launches
+        achieved = gemm_flops[name] / (avg_ms / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": name,
+                "avg_launch_ms": avg_ms,
+                "peak_source": f"{pk['source']} bf16 sustained (kernel timed inside a long step)"}
+    launches_total = sum(v[0] for v in kt.values())
+    kernel_table = {kname: {"launches": v[0], "ms_per_launch": v[1] / v[0],
+                            "share": v[1] / sum(u[1] for u in kt.values())} for kname, v in kt.items()}
+    if args.kernel_table:
+        for kname, v in sorted(kernel_table.items(), key=lambda kv: -kv[1]["share"]):
+            sys.stderr.write(f"{kname:24s} {v['launches']:5d} {v['ms_per_launch']:9.4f} ms {100 * v['share']:5.1f}%\n")
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        n_tok = 64
+        n, dt = oracle_sample(wl, args.seed, n_tok, inp)
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"first {n} tokens of the {wl.name} batch, fwd+bwd, fp64 numpy "
+                         f"({dt:.1f} s)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random MXFP4 codes, UE8M0 scales 119..123)",
+        "config": {"workload": wl.name, "T": T, "H": H, "I": I, "E": E, "k": k,
+                   "tokens_per_gpu": T, "l2": "inputs larger than L2 (423 MB of packed weights "
+                   "and ~1.5 GB of per-step activations)",
+                   "tflops": flop_step * world * args.steps / (ms_max / 1e3) / 1e12,
+                   "tensor_frac_of_sustained": flop_step * world * args.steps / (ms_max / 1e3) / 1e12
+                   / pk["bf16_tflops_sustained"]},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": T * world * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_total,
+        "kernels": kernel_table,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

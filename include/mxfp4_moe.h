@@ -1,0 +1,185 @@
+/*
+ * mxfp4_moe.h -- C ABI of the MXFP4 mixture-of-experts expert block on NVIDIA B200 (sm_100a).
+ *
+ * What it computes
+ * ----------------
+ * The expert block of a GPT-OSS-style MoE layer whose expert weights stay packed as MXFP4,
+ * forward and input-gradient backward, for adapter (LoRA) training where the quantized base
+ * is frozen.  Sources:
+ *   - "Add MXFP4 training support via a dequantize-on-the-fly fallback" (huggingface/
+ *     transformers #47464), section "What this does": top-k router plus a GptOssExperts-style
+ *     expert loop over weights dequantized on the fly, packed storage never modified; section
+ *     "Relation to the backward triton kernels": gradients must reach the inputs through the
+ *     expert math, the frozen base never needs a weight gradient.
+ *   - "Integrate finegrained kernels: SOTA performance and per-module quantization"
+ *     (huggingface/transformers #49658), commit on the gate|up row interleave (gate j at row
+ *     2j, up j at row 2j+1; the GLU splits with stride 2) and commit on the per-expert bias
+ *     operand (bias indexed by the tile's expert id, on the same output-row axis as the
+ *     weight, fused in both GEMMs; the host keeps only the routing-weighted reduce).
+ *   - OCP Microscaling Formats (MX) v1.0: E2M1 elements, UE8M0 scales (2^(s-127), 255 = NaN),
+ *     32 elements per scale.
+ *
+ * Notation: T tokens, H hidden size, I intermediate size, E experts, k experts per token,
+ * A = T*k (token, slot) assignments.  Forward per token t with selected experts e_j, j < k:
+ *     w_t       = softmax over the k largest logits (largest first, ties -> lower index)
+ *     h_{t,j}   = x_t W_gu[e_j]^T + b_gu[e_j]                       (2I, interleaved g/u)
+ *     a_{t,j}   = (min(max(u,-L),L) + 1) * min(g,L) * sigmoid(alpha*min(g,L))   (I)
+ *     y_{t,j}   = a_{t,j} W_d[e_j]^T + b_d[e_j]                      (H)
+ *     out_t     = sum_j w_{t,j} y_{t,j}
+ * Backward (given dY = dL/d out): dX = dL/dx, d_topk_w[t,j] = <dY_t, y_{t,j}>, and
+ * d_logits = softmax-over-k Jacobian applied to d_topk_w (zero for unselected experts).
+ * No weight gradient.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major, densely packed,
+ *    at least 16-byte aligned.  "bf16" buffers are uint16_t bit patterns.  The library never
+ *    allocates or frees device memory and never synchronizes the stream, except
+ *    mxfp4_moe_check.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Work is
+ *    enqueued on it and the call returns; results are valid once the stream reaches them.
+ *  - Return value: 0 on success, a negative MXFP4_MOE_ERR_* code otherwise.  Argument errors
+ *    are detected before anything is enqueued.  Faults detected on the device (a bounded wait
+ *    that expired, an index out of range) are written to an error word inside the workspace
+ *    and reported by mxfp4_moe_check.
+ *  - The current CUDA device must be an sm_100 part (B200); otherwise
+ *    MXFP4_MOE_ERR_UNSUPPORTED_DEVICE.
+ *  - Shapes: H and I multiples of 32 (one MX block), 1 <= k <= E <= 256, T >= 1, A = T*k < 2^31.
+ */
+#ifndef MXFP4_MOE_H_
+#define MXFP4_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MXFP4_MOE_API __attribute__((visibility("default")))
+#else
+#define MXFP4_MOE_API
+#endif
+
+#define MXFP4_MOE_OK 0
+#define MXFP4_MOE_ERR_INVALID_ARG (-1)         /* null pointer, bad shape, misaligned pointer */
+#define MXFP4_MOE_ERR_WORKSPACE_TOO_SMALL (-2)  /* ws_bytes below mxfp4_moe_workspace_size  */
+#define MXFP4_MOE_ERR_UNSUPPORTED_DEVICE (-3)   /* current device is not sm_100           */
+#define MXFP4_MOE_ERR_CUDA (-4)                 /* a CUDA runtime call or launch failed    */
+#define MXFP4_MOE_ERR_DEVICE_TIMEOUT (-5)       /* a bounded device-side wait expired      */
+#define MXFP4_MOE_ERR_DEVICE_BOUNDS (-6)        /* a device-side index check failed        */
+
+/* Problem shape and GLU constants (GPT-OSS: glu_alpha = 1.702, glu_limit = 7). */
+typedef struct {
+  int32_t T, H, I, E, k;
+  float glu_alpha;
+  float glu_limit;
+} mxfp4_moe_dims;
+
+/* Frozen expert weights in the packed MXFP4 layout (read only, never modified).
+ *   gu_blocks  uint8 [E][2I][H/2]  gate_up rows, interleaved: row 2j = gate j, row 2j+1 = up j.
+ *                                  Byte i of a row holds element 2i (low nibble) and 2i+1
+ *                                  (high nibble), E2M1 codes.
+ *   gu_scales  uint8 [E][2I][H/32] UE8M0 scale of each 32-element block of a row.
+ *   gu_bias    bf16  [E][2I]       interleaved like the rows.
+ *   dn_blocks  uint8 [E][H][I/2]   down rows, same packing along I.
+ *   dn_scales  uint8 [E][H][I/32]
+ *   dn_bias    bf16  [E][H]
+ * Stacked [gate; up] checkpoints must be interleaved by the caller first; the bytes do not
+ * tell the two orders apart. */
+typedef struct {
+  const uint8_t* gu_blocks;
+  const uint8_t* gu_scales;
+  const uint16_t* gu_bias;
+  const uint8_t* dn_blocks;
+  const uint8_t* dn_scales;
+  const uint16_t* dn_bias;
+} mxfp4_moe_weights;
+
+/* Bytes of device workspace that mxfp4_moe_forward / mxfp4_moe_backward_input need for `d`.
+ * The forward leaves its saved state (routing, permutation, gate_up pre-activations) in the
+ * workspace; the backward reads it and uses the rest as scratch.
+ * Errors: INVALID_ARG (null pointers, bad shape). */
+MXFP4_MOE_API int mxfp4_moe_workspace_size(const mxfp4_moe_dims* d, size_t* bytes);
+
+/* Bytes of the transposed weight copy made by mxfp4_moe_transpose_weights. */
+MXFP4_MOE_API int mxfp4_moe_transposed_weights_size(const mxfp4_moe_dims* d, size_t* bytes);
+
+/* One-time layout step for the backward (weights are frozen, so it is done once per set of
+ * weights, not per step).  The input-gradient GEMMs contract over the OUTPUT axis of the
+ * stored weights (dact = dy W_d, dx = dh W_gu), where the 32-element scale blocks run across
+ * the contraction.  This call writes the same E2M1 codes and UE8M0 scale bytes, transposed:
+ *   [0, E*I*H/2)           dn_blocks_t uint8 [E][I][H/2]   element (i, h) = W_d[e][h][i]
+ *   then E*(2I)*H/2 bytes  gu_blocks_t uint8 [E][H][2I/2]  element (h, n) = W_gu[e][n][h]
+ *   then E*(I/32)*H bytes  dn_scales_t uint8 [E][I/32][H]  = dn_scales[e][h][i/32]
+ *   then E*(H/32)*2I bytes gu_scales_t uint8 [E][H/32][2I] = gu_scales[e][n][h/32]
+ * (each region starts 256-byte aligned).  Values are not re-quantized; the copy is still
+ * packed MXFP4 (4.25 bits per weight).
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL (wt_bytes too small), UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_transpose_weights(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, void* wt,
+                                size_t wt_bytes, void* stream);
+
+/* Forward.
+ *   x        bf16  [T][H]   activations
+ *   logits   fp32  [T][E]   router logits (the router linear stays with the caller)
+ *   y        bf16  [T][H]   output: sum_j w_{t,j} y_{t,j}
+ *   topk_idx int32 [T][k]   output, may be NULL: selected experts, largest logit first
+ *   topk_w   fp32  [T][k]   output, may be NULL: softmax over the selected logits
+ *   ws, ws_bytes            workspace (>= mxfp4_moe_workspace_size); keep it unmodified until
+ *                           mxfp4_moe_backward_input has been enqueued if a backward follows.
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const uint16_t* x,
+                      const float* logits, uint16_t* y, int32_t* topk_idx, float* topk_w,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Input-gradient backward through the frozen quantized weights (no weight gradient).
+ *   wt       the transposed copy from mxfp4_moe_transpose_weights for the same weights
+ *   dy       bf16 [T][H]  upstream gradient dL/d(out)
+ *   ws       the workspace the matching mxfp4_moe_forward used (its saved state is read; the
+ *            scratch part is overwritten)
+ *   dx       bf16 [T][H]  output dL/dx
+ *   d_topk_w fp32 [T][k]  output dL/d(topk_w), slot order of the forward's topk_idx
+ *   d_logits fp32 [T][E]  output, may be NULL: dL/d(logits) through the softmax over k
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w,
+                             const void* wt, size_t wt_bytes, const uint16_t* dy, void* ws,
+                             size_t ws_bytes, uint16_t* dx, float* d_topk_w, float* d_logits,
+                             void* stream);
+
+/* Standalone dequantization (diagnostics and tests): rows of packed MXFP4 -> bf16.
+ *   blocks uint8 [rows][K/2], scales uint8 [rows][K/32], out bf16 [rows][K]; K multiple of 32.
+ * out = bf16(E2M1(code) * 2^(s-127)), exact (the product is always representable in bf16 or
+ * overflows to inf); s = 255 gives NaN.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
+                         uint16_t* out, void* stream);
+
+/* Synchronize `stream`, then read and clear the device error word in `ws` (a workspace used by
+ * forward/backward).  Returns 0, DEVICE_TIMEOUT or DEVICE_BOUNDS (from the device), or CUDA
+ * if the stream reported an error.  `where` (may be NULL) receives the device-side tag. */
+MXFP4_MOE_API int mxfp4_moe_check(void* ws, void* stream, int32_t* where);
+
+/* Per-kernel timing (diagnostics).  Between mxfp4_moe_profile_begin() and
+ * mxfp4_moe_profile_end(), the library records a CUDA event pair on the launching stream around
+ * every kernel it enqueues (host-side bookkeeping only; results are unchanged).
+ * mxfp4_moe_profile_end synchronizes those events and fills up to `max` entries of `out` with
+ * one line per kernel name: launches and summed device time in milliseconds; `*n` receives the
+ * number of distinct kernels.  Not thread-safe: profile from one host thread.
+ * Errors: INVALID_ARG (null out/n), CUDA. */
+typedef struct {
+  char name[48];
+  int32_t launches;
+  double total_ms;
+} mxfp4_moe_kernel_time;
+MXFP4_MOE_API int mxfp4_moe_profile_begin(void);
+MXFP4_MOE_API int mxfp4_moe_profile_end(mxfp4_moe_kernel_time* out, int32_t max, int32_t* n);
+
+/* Static description of a return code. */
+MXFP4_MOE_API const char* mxfp4_moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXFP4_MOE_H_ */

@@ -1,0 +1,359 @@
+// C ABI of the MXFP4 MoE expert block: argument checks, workspace carving and the launch
+// sequence of the forward and input-gradient backward.  See include/mxfp4_moe.h.
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "../../include/mxfp4_moe.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+  size_t err, hist, off, idx, w, perm, inv, h, act_dh, rows, cbias, dwp, total;
+};
+
+WsLayout ws_layout(const mxfp4_moe_dims& d) {
+  const size_t A = (size_t)d.T * d.k;
+  WsLayout L{};
+  size_t o = 0;
+  L.err = o;    o = up(o + 16);
+  L.hist = o;   o = up(o + 4ull * d.E);
+  L.off = o;    o = up(o + 4ull * (d.E + 1));
+  L.idx = o;    o = up(o + 4 * A);
+  L.w = o;      o = up(o + 4 * A);
+  L.perm = o;   o = up(o + 4 * A);
+  L.inv = o;    o = up(o + 4 * A);
+  L.h = o;      o = up(o + 2 * A * 2 * d.I);   // saved gate_up pre-activations
+  L.act_dh = o; o = up(o + 2 * A * 2 * d.I);   // act [A][I] (fwd) / dH [A][2I] (bwd)
+  L.rows = o;   o = up(o + 2 * A * d.H);       // Xp/Yslot (fwd), dYp/dXslot (bwd)
+  L.cbias = o;  o = up(o + 4 * A);
+  L.dwp = o;    o = up(o + 4 * A * (d.I / 32));
+  L.total = o;
+  return L;
+}
+
+struct WtLayout {
+  size_t dn_blocks, gu_blocks, dn_scales, gu_scales, total;
+};
+
+WtLayout wt_layout(const mxfp4_moe_dims& d) {
+  WtLayout L{};
+  const size_t E = d.E, H = d.H, I = d.I;
+  size_t o = 0;
+  L.dn_blocks = o; o = up(o + E * I * (H / 2));
+  L.gu_blocks = o; o = up(o + E * H * I);
+  L.dn_scales = o; o = up(o + E * (I / 32) * H);
+  L.gu_scales = o; o = up(o + E * (H / 32) * 2 * I);
+  L.total = o;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const mxfp4_moe_dims* d) {
+  if (!d) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (d->T < 1 || d->H < 32 || d->I < 32 || d->H % 32 || d->I % 32) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (d->E < 1 || d->E > 256 || d->k < 1 || d->k > d->E) return MXFP4_MOE_ERR_INVALID_ARG;
+  if ((long long)d->T * d->k >= (1ll << 31)) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (!(d->glu_limit > 0.f) || !(d->glu_alpha == d->glu_alpha)) return MXFP4_MOE_ERR_INVALID_ARG;
+  // the grouped GEMM keeps a tile's scales for the whole contraction in shared memory
+  if (moe::grouped_gemm_smem_bytes(d->H > 2 * d->I ? d->H : 2 * d->I) > 232448)
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  return MXFP4_MOE_OK;
+}
+
+int check_weights(const mxfp4_moe_weights* w) {
+  if (!w || !w->gu_blocks || !w->gu_scales || !w->gu_bias || !w->dn_blocks || !w->dn_scales ||
+      !w->dn_bias)
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->gu_blocks) || !aligned16(w->gu_scales) || !aligned16(w->dn_blocks) ||
+      !aligned16(w->dn_scales) || !aligned16(w->gu_bias) || !aligned16(w->dn_bias))
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  return MXFP4_MOE_OK;
+}
+
+// Current device must be sm_100 (B200).  Returns the SM count through `sms`.
+int check_device(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MXFP4_MOE_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return MXFP4_MOE_ERR_CUDA;
+  if (major != 10 || minor != 0) return MXFP4_MOE_ERR_UNSUPPORTED_DEVICE;
+  if (sms && cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MXFP4_MOE_ERR_CUDA;
+  return MXFP4_MOE_OK;
+}
+
+#define MOE_TRY(expr)                                  \
+  do {                                                 \
+    cudaError_t e_ = (expr);                           \
+    if (e_ != cudaSuccess) return MXFP4_MOE_ERR_CUDA;  \
+  } while (0)
+
+template <class T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+
+// ---- per-kernel event timing (mxfp4_moe_profile_begin / _end) -------------------------
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+
+// Brackets one kernel launch with an event pair when profiling is on.
+struct Timed {
+  const char* name;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  Timed(const char* n, cudaStream_t s) : name(n), st(s) {
+    if (prof().on) {
+      a = prof().get();
+      cudaEventRecord(a, st);
+    }
+  }
+  ~Timed() {
+    if (a) {
+      cudaEvent_t b = prof().get();
+      cudaEventRecord(b, st);
+      prof().recs.push_back({name, a, b});
+    }
+  }
+};
+
+#define MOE_LAUNCH(name, expr)   \
+  do {                           \
+    Timed timed_(name, st);      \
+    MOE_TRY(expr);               \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int mxfp4_moe_workspace_size(const mxfp4_moe_dims* d, size_t* bytes) {
+  const int rc = check_dims(d);
+  if (rc) return rc;
+  if (!bytes) return MXFP4_MOE_ERR_INVALID_ARG;
+  *bytes = ws_layout(*d).total;
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_transposed_weights_size(const mxfp4_moe_dims* d, size_t* bytes) {
+  const int rc = check_dims(d);
+  if (rc) return rc;
+  if (!bytes) return MXFP4_MOE_ERR_INVALID_ARG;
+  *bytes = wt_layout(*d).total;
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_transpose_weights(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, void* wt,
+                                size_t wt_bytes, void* stream) {
+  int rc = check_dims(d);
+  if (!rc) rc = check_weights(w);
+  if (rc) return rc;
+  if (!wt || !aligned16(wt)) return MXFP4_MOE_ERR_INVALID_ARG;
+  const WtLayout L = wt_layout(*d);
+  if (wt_bytes < L.total) return MXFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
+  rc = check_device(nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_LAUNCH("transpose_packed", moe::launch_transpose_packed(w->dn_blocks, d->E, d->H, d->I, at<uint8_t>(wt, L.dn_blocks), st));
+  MOE_LAUNCH("transpose_packed", moe::launch_transpose_packed(w->gu_blocks, d->E, 2 * d->I, d->H, at<uint8_t>(wt, L.gu_blocks), st));
+  MOE_LAUNCH("transpose_scales", moe::launch_transpose_scales(w->dn_scales, d->E, d->H, d->I, at<uint8_t>(wt, L.dn_scales), st));
+  MOE_LAUNCH("transpose_scales", moe::launch_transpose_scales(w->gu_scales, d->E, 2 * d->I, d->H, at<uint8_t>(wt, L.gu_scales), st));
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const uint16_t* x,
+                      const float* logits, uint16_t* y, int32_t* topk_idx, float* topk_w,
+                      void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(d);
+  if (!rc) rc = check_weights(w);
+  if (rc) return rc;
+  if (!x || !logits || !y || !ws || !aligned16(x) || !aligned16(y) || !aligned16(ws) ||
+      (reinterpret_cast<uintptr_t>(logits) & 3u))
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*d);
+  if (ws_bytes < L.total) return MXFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  rc = check_device(&sms);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->k, A = T * k;
+  int* err = at<int>(ws, L.err);
+  int32_t* hist = at<int32_t>(ws, L.hist);
+  int32_t* off = at<int32_t>(ws, L.off);
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* wr = at<float>(ws, L.w);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  uint16_t* h = at<uint16_t>(ws, L.h);
+  uint16_t* act = at<uint16_t>(ws, L.act_dh);
+  uint16_t* rows = at<uint16_t>(ws, L.rows);
+
+  MOE_TRY(cudaMemsetAsync(hist, 0, 4ull * E, st));
+  MOE_LAUNCH("router_topk", moe::launch_router_topk(logits, T, E, k, idx, wr, hist, topk_idx, topk_w, err, st));
+  MOE_LAUNCH("build_perm", moe::launch_build_perm(idx, A, E, hist, off, perm, inv, err, st));
+  MOE_LAUNCH("gather_x", moe::launch_gather_rows(x, H, k, perm, A, rows, off, E, nullptr, nullptr, st));
+
+  moe::GemmArgs g{};
+  g.off = off; g.E = E; g.A = A; g.perm = perm; g.topk_w = wr; g.err = err;
+  g.alpha = d->glu_alpha; g.limit = d->glu_limit;
+  // gate_up: h = Xp W_gu^T + b_gu, act = GLU(h)
+  g.scales = w->gu_scales; g.K = H; g.N = 2 * I; g.bias = w->gu_bias; g.out0 = h; g.out1 = act;
+  MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, rows, w->gu_blocks, g, sms, st));
+  // down: Yslot[slot] = w_slot * (act W_d^T + b_d)
+  g.scales = w->dn_scales; g.K = I; g.N = H; g.bias = w->dn_bias; g.out0 = rows; g.out1 = nullptr;
+  MOE_LAUNCH("gemm_down_scatter", moe::launch_grouped_gemm(moe::kEpiDown, false, act, w->dn_blocks, g, sms, st));
+  MOE_LAUNCH("combine_y", moe::launch_combine(rows, T, k, H, y, st));
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w,
+                             const void* wt, size_t wt_bytes, const uint16_t* dy, void* ws,
+                             size_t ws_bytes, uint16_t* dx, float* d_topk_w, float* d_logits,
+                             void* stream) {
+  int rc = check_dims(d);
+  if (!rc) rc = check_weights(w);
+  if (rc) return rc;
+  if (!wt || !dy || !ws || !dx || !d_topk_w || !aligned16(wt) || !aligned16(dy) ||
+      !aligned16(ws) || !aligned16(dx) || !aligned16(d_topk_w) ||
+      (d_logits && !aligned16(d_logits)))
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*d);
+  const WtLayout LT = wt_layout(*d);
+  if (ws_bytes < L.total || wt_bytes < LT.total) return MXFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  rc = check_device(&sms);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->k, A = T * k;
+  void* wtp = const_cast<void*>(wt);
+  int* err = at<int>(ws, L.err);
+  int32_t* off = at<int32_t>(ws, L.off);
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* wr = at<float>(ws, L.w);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  uint16_t* h = at<uint16_t>(ws, L.h);
+  uint16_t* dh = at<uint16_t>(ws, L.act_dh);
+  uint16_t* rows = at<uint16_t>(ws, L.rows);
+  float* cbias = at<float>(ws, L.cbias);
+  float* dwp = at<float>(ws, L.dwp);
+
+  // dYp[row] = dY[t(row)], cbias[row] = <dY[t], b_d[e(row)]>
+  MOE_LAUNCH("gather_dy_bias_dot", moe::launch_gather_rows(dy, H, k, perm, A, rows, off, E, w->dn_bias, cbias, st));
+  moe::GemmArgs g{};
+  g.off = off; g.E = E; g.A = A; g.perm = perm; g.topk_w = wr; g.err = err;
+  g.alpha = d->glu_alpha; g.limit = d->glu_limit;
+  // dZ = dYp W_d (contract over H); epilogue: GLU derivative -> dH, partial <dZ, act>
+  g.scales = at<uint8_t>(wtp, LT.dn_scales); g.K = H; g.N = I; g.out0 = dh; g.hsaved = h;
+  g.dw_part = dwp;
+  MOE_LAUNCH("gemm_dact_glu_bwd", moe::launch_grouped_gemm(moe::kEpiDact, true, rows, at<uint8_t>(wtp, LT.dn_blocks), g, sms, st));
+  // dx = dH W_gu (contract over the 2I interleaved rows)
+  g.scales = at<uint8_t>(wtp, LT.gu_scales); g.K = 2 * I; g.N = H; g.out0 = rows; g.hsaved = nullptr;
+  g.dw_part = nullptr;
+  MOE_LAUNCH("gemm_dx_scatter", moe::launch_grouped_gemm(moe::kEpiDx, true, dh, at<uint8_t>(wtp, LT.gu_blocks), g, sms, st));
+  MOE_LAUNCH("combine_dx", moe::launch_combine(rows, T, k, H, dx, st));
+  MOE_LAUNCH("router_backward", moe::launch_router_backward(idx, wr, inv, cbias, dwp, I / 32, T, E, k, d_topk_w, d_logits, st));
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
+                         uint16_t* out, void* stream) {
+  if (!blocks || !scales || !out || rows < 0 || K < 32 || K % 32 || !aligned16(blocks) ||
+      !aligned16(out))
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  const int rc = check_device(nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_LAUNCH("dequant", moe::launch_dequant(blocks, scales, rows, K, out, st));
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_check(void* ws, void* stream, int32_t* where) {
+  if (!ws) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MXFP4_MOE_ERR_CUDA;
+  int word[2] = {0, 0};
+  if (cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MXFP4_MOE_ERR_CUDA;
+  if (word[0] != 0 && cudaMemset(ws, 0, sizeof(word)) != cudaSuccess) return MXFP4_MOE_ERR_CUDA;
+  if (where) *where = word[1];
+  return word[0];
+}
+
+int mxfp4_moe_profile_begin(void) {
+  prof().on = true;
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_profile_end(mxfp4_moe_kernel_time* out, int32_t max, int32_t* n) {
+  if (!out || !n || max < 0) return MXFP4_MOE_ERR_INVALID_ARG;
+  Profiler& P = prof();
+  P.on = false;
+  int rc = MXFP4_MOE_OK;
+  int cnt = 0;
+  for (const ProfRec& r : P.recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+      rc = MXFP4_MOE_ERR_CUDA;
+    int i = 0;
+    while (i < cnt && i < max && std::strncmp(out[i].name, r.name, sizeof(out[i].name)) != 0) ++i;
+    if (i == cnt && cnt < max) {
+      std::memset(&out[i], 0, sizeof(out[i]));
+      std::strncpy(out[i].name, r.name, sizeof(out[i].name) - 1);
+      ++cnt;
+    }
+    if (i < cnt) {
+      out[i].launches += 1;
+      out[i].total_ms += ms;
+    }
+    P.pool.push_back(r.a);
+    P.pool.push_back(r.b);
+  }
+  P.recs.clear();
+  *n = cnt;
+  return rc;
+}
+
+const char* mxfp4_moe_strerror(int code) {
+  switch (code) {
+    case MXFP4_MOE_OK: return "ok";
+    case MXFP4_MOE_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or unsupported shape)";
+    case MXFP4_MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than the size query returned";
+    case MXFP4_MOE_ERR_UNSUPPORTED_DEVICE: return "current CUDA device is not sm_100 (B200)";
+    case MXFP4_MOE_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case MXFP4_MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    case MXFP4_MOE_ERR_DEVICE_BOUNDS: return "a device-side index check failed";
+    default: return "unknown error code";
+  }
+}
+
+}  // extern "C"

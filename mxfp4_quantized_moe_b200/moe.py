@@ -1,0 +1,154 @@
+"""Torch-facing wrappers over the C ABI (device memory and streams come from torch).
+
+Each function checks shapes and dtypes, hands raw device pointers and the current CUDA
+stream to the library, and returns torch tensors.  All computation happens in the
+library's kernels.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import Dims, Weights, check, lib
+
+
+@dataclass
+class MoeShape:
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    glu_alpha: float = 1.702
+    glu_limit: float = 7.0
+
+    def dims(self) -> Dims:
+        return Dims(self.T, self.H, self.I, self.E, self.k, self.glu_alpha, self.glu_limit)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _weights(w: dict) -> Weights:
+    for key, dt in (("gu_blocks", torch.uint8), ("gu_scales", torch.uint8),
+                    ("gu_bias", torch.bfloat16), ("dn_blocks", torch.uint8),
+                    ("dn_scales", torch.uint8), ("dn_bias", torch.bfloat16)):
+        if w[key].dtype != dt:
+            raise TypeError(f"{key} must be {dt}")
+    return Weights(_ptr(w["gu_blocks"]), _ptr(w["gu_scales"]), _ptr(w["gu_bias"]),
+                   _ptr(w["dn_blocks"]), _ptr(w["dn_scales"]), _ptr(w["dn_bias"]))
+
+
+def workspace_bytes(shape: MoeShape) -> int:
+    n = ctypes.c_size_t()
+    check(lib.mxfp4_moe_workspace_size(ctypes.byref(shape.dims()), ctypes.byref(n)),
+          "mxfp4_moe_workspace_size")
+    return n.value
+
+
+def transposed_weights_bytes(shape: MoeShape) -> int:
+    n = ctypes.c_size_t()
+    check(lib.mxfp4_moe_transposed_weights_size(ctypes.byref(shape.dims()), ctypes.byref(n)),
+          "mxfp4_moe_transposed_weights_size")
+    return n.value
+
+
+def alloc_workspace(shape: MoeShape, device="cuda") -> torch.Tensor:
+    return torch.zeros(workspace_bytes(shape), dtype=torch.uint8, device=device)
+
+
+def transpose_weights(shape: MoeShape, w: dict, out: torch.Tensor | None = None, stream=None):
+    n = transposed_weights_bytes(shape)
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=w["gu_blocks"].device)
+    check(lib.mxfp4_moe_transpose_weights(ctypes.byref(shape.dims()), ctypes.byref(_weights(w)),
+                                          _ptr(out), out.numel(), _stream(stream)),
+          "mxfp4_moe_transpose_weights")
+    return out
+
+
+def forward(shape: MoeShape, w: dict, x: torch.Tensor, logits: torch.Tensor, ws: torch.Tensor,
+            y: torch.Tensor | None = None, topk_idx: torch.Tensor | None = None,
+            topk_w: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    T, H = shape.T, shape.H
+    if x.shape != (T, H) or x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16 [T, H]")
+    if logits.shape != (T, shape.E) or logits.dtype != torch.float32:
+        raise ValueError("logits must be fp32 [T, E]")
+    if y is None:
+        y = torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
+    check(lib.mxfp4_moe_forward(ctypes.byref(shape.dims()), ctypes.byref(_weights(w)), _ptr(x),
+                                _ptr(logits), _ptr(y), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
+                                ws.numel(), _stream(stream)), "mxfp4_moe_forward")
+    return y
+
+
+def backward_input(shape: MoeShape, w: dict, wt: torch.Tensor, dy: torch.Tensor,
+                   ws: torch.Tensor, dx: torch.Tensor | None = None,
+                   d_topk_w: torch.Tensor | None = None, d_logits: torch.Tensor | None = None,
+                   want_d_logits: bool = True, stream=None):
+    T, H = shape.T, shape.H
+    if dy.shape != (T, H) or dy.dtype != torch.bfloat16:
+        raise ValueError("dy must be bf16 [T, H]")
+    dev = dy.device
+    if dx is None:
+        dx = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    if d_topk_w is None:
+        d_topk_w = torch.empty(T, shape.k, dtype=torch.float32, device=dev)
+    if d_logits is None and want_d_logits:
+        d_logits = torch.empty(T, shape.E, dtype=torch.float32, device=dev)
+    check(lib.mxfp4_moe_backward_input(ctypes.byref(shape.dims()), ctypes.byref(_weights(w)),
+                                       _ptr(wt), wt.numel(), _ptr(dy), _ptr(ws), ws.numel(),
+                                       _ptr(dx), _ptr(d_topk_w), _ptr(d_logits),
+                                       _stream(stream)), "mxfp4_moe_backward_input")
+    return dx, d_topk_w, d_logits
+
+
+def dequantize(blocks: torch.Tensor, scales: torch.Tensor, stream=None) -> torch.Tensor:
+    """bf16 [rows, K] from packed uint8 [rows, K/2] and UE8M0 scales [rows, K/32]."""
+    rows = blocks.numel() // blocks.shape[-1]
+    K = blocks.shape[-1] * 2
+    if scales.numel() != rows * (K // 32):
+        raise ValueError("scales do not match blocks")
+    out = torch.empty(*blocks.shape[:-1], K, dtype=torch.bfloat16, device=blocks.device)
+    check(lib.mxfp4_moe_dequantize(_ptr(blocks), _ptr(scales), rows, K, _ptr(out),
+                                   _stream(stream)), "mxfp4_moe_dequantize")
+    return out
+
+
+def device_check(ws: torch.Tensor, stream=None) -> tuple[int, int]:
+    """Synchronize and read (then clear) the device error word: (code, where)."""
+    where = ctypes.c_int32(0)
+    rc = lib.mxfp4_moe_check(_ptr(ws), _stream(stream), ctypes.byref(where))
+    return rc, where.value
+
+
+def weights_to(inp: dict, device) -> dict:
+    keys = ("gu_blocks", "gu_scales", "gu_bias", "dn_blocks", "dn_scales", "dn_bias")
+    return {k: inp[k].to(device).contiguous() for k in keys}
+
+
+def profile_begin() -> None:
+    check(lib.mxfp4_moe_profile_begin(), "mxfp4_moe_profile_begin")
+
+
+def profile_end() -> dict:
+    """{kernel name: (launches, total device ms)} since profile_begin()."""
+    buf = (_lib.KernelTime * 64)()
+    n = ctypes.c_int32(0)
+    check(lib.mxfp4_moe_profile_end(buf, 64, ctypes.byref(n)), "mxfp4_moe_profile_end")
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(n.value)}

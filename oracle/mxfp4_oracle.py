@@ -34,7 +34,11 @@ Readings where the pages are silent (each pinned by a test):
   softmax over the k selected logits; slot j of a token holds its j-th largest;
 * bias placement: added before the GLU clamp (gate_up) and before the routing
   weight multiply (down), so the routing weight scales the down bias too;
-* clamp derivative: inclusive mask (gradient passes at g == limit, |u| == limit).
+* clamp derivative: inclusive mask (gradient passes at g == limit, |u| == limit),
+  decided on the gate_up pre-activation rounded to bf16.  The eager reference runs the
+  GPT-OSS expert loop on bf16 tensors (its dequantized transients are bf16), so autograd's
+  clamp backward sees h as a bf16 tensor; the mask is a yes/no decision and is taken in
+  that precision.  Everything else stays fp64.
 """
 
 from __future__ import annotations
@@ -128,6 +132,11 @@ def _f64_to_bf16_bits(x):
     return out.astype(np.uint16)
 
 
+def round_bf16(x) -> np.ndarray:
+    """fp64 values rounded to the nearest bf16 (ties to even), as fp64."""
+    return bf16_bits_to_f64(f64_to_bf16_bits(x))
+
+
 def bf16_bits_to_f64(bits) -> np.ndarray:
     """16-bit bf16 patterns -> fp64 values (exact)."""
     b = np.asarray(bits, dtype=np.int64) & 0xFFFF
@@ -178,19 +187,26 @@ def glu(h, alpha: float = 1.702, limit: float = 7.0):
     return (uc + 1.0) * gc * _sigmoid(alpha * gc)
 
 
-def glu_backward(h, dact, alpha: float = 1.702, limit: float = 7.0):
-    """d(act)/d(h) applied to dact; returns dh with the same interleaved layout as h."""
+def glu_backward(h, dact, alpha: float = 1.702, limit: float = 7.0, h_mask=None):
+    """d(act)/d(h) applied to dact; returns dh with the same interleaved layout as h.
+
+    The clamps pass the gradient where g <= limit and -limit <= u <= limit (inclusive).
+    ``h_mask`` (default: h) is the tensor those two decisions are taken on.
+    """
     h = np.asarray(h, dtype=np.float64)
     dact = np.asarray(dact, dtype=np.float64)
+    hm = h if h_mask is None else np.asarray(h_mask, dtype=np.float64)
     g = h[..., 0::2]
     u = h[..., 1::2]
+    gm = hm[..., 0::2]
+    um = hm[..., 1::2]
     gc = np.minimum(g, limit)
     uc = np.clip(u, -limit, limit)
     s = _sigmoid(alpha * gc)
     d_gc = (uc + 1.0) * (s + alpha * gc * s * (1.0 - s))
     d_uc = gc * s
-    dg = dact * d_gc * (g <= limit)
-    du = dact * d_uc * ((u >= -limit) & (u <= limit))
+    dg = dact * d_gc * (gm <= limit)
+    du = dact * d_uc * ((um >= -limit) & (um <= limit))
     dh = np.empty(h.shape, dtype=np.float64)
     dh[..., 0::2] = dg
     dh[..., 1::2] = du
@@ -259,7 +275,9 @@ def moe_backward(dY, fwd, W, alpha: float = 1.702, limit: float = 7.0):
         wgu, wd = _expert_weights(W, e)
         dy = w[tt, jj][:, None] * dY[tt]
         dact = dy @ wd  # [n, I]
-        dh = glu_backward(fwd["h"][tt, jj], dact, alpha, limit)  # [n, 2I]
+        h = fwd["h"][tt, jj]
+        # clamp masks decided on the pre-activation as the eager bf16 model holds it
+        dh = glu_backward(h, dact, alpha, limit, h_mask=round_bf16(h))  # [n, 2I]
         dx = dh @ wgu  # [n, H]
         np.add.at(dX, tt, dx)
     d_w = np.einsum("th,tjh->tj", dY, fwd["y"])

@@ -57,6 +57,14 @@ def _topk(row, k):
     return chosen
 
 
+def _bf16(v: float) -> float:
+    """Round to the nearest bf16 (8 significant bits, ties to even); normal range only."""
+    if v == 0.0 or math.isinf(v) or math.isnan(v):
+        return v
+    m, e = math.frexp(v)  # v = m * 2^e, 0.5 <= |m| < 1
+    return math.ldexp(round(m * 256.0), e - 8)  # Python round() is half-to-even
+
+
 def _sig(z):
     return 1.0 / (1.0 + math.exp(-z))
 
@@ -100,8 +108,9 @@ def forward_backward(x, logits, dY, W, k, alpha=1.702, limit=7.0):
                 act.append((uc + 1.0) * gc * s)
                 dgc.append((uc + 1.0) * (s + alpha * gc * s * (1.0 - s)))
                 duc.append(gc * s)
-                gm.append(1.0 if g <= limit else 0.0)
-                um.append(1.0 if -limit <= u <= limit else 0.0)
+                gb, ub = _bf16(g), _bf16(u)  # clamp masks decided on bf16 pre-activations
+                gm.append(1.0 if gb <= limit else 0.0)
+                um.append(1.0 if -limit <= ub <= limit else 0.0)
             y = [sum(act[i] * wd[hh][i] for i in range(I)) + bd[hh] for hh in range(H)]
             for hh in range(H):
                 o[hh] += w[j] * y[hh]

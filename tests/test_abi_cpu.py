@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol the
+header declares, and validates arguments before touching a device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxfp4_moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from mxfp4_quantized_moe_b200 import build
+    build.build()
+    from mxfp4_quantized_moe_b200 import _lib
+    return _lib
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return re.findall(r"MXFP4_MOE_API\s+[\w\s\*]+?\b(mxfp4_moe_\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for must in ("mxfp4_moe_forward", "mxfp4_moe_backward_input", "mxfp4_moe_workspace_size",
+                 "mxfp4_moe_transpose_weights", "mxfp4_moe_dequantize", "mxfp4_moe_check",
+                 "mxfp4_moe_strerror"):
+        assert must in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    lib = ctypes.CDLL(L.LIB_PATH)
+    syms = declared_symbols()
+    assert syms
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) == set(L.SIGNATURES)
+
+
+def test_error_codes_match_header(L):
+    src = open(HEADER).read()
+    codes = dict(re.findall(r"#define (MXFP4_MOE_\w+) \(?(-?\d+)\)?", src))
+    assert int(codes["MXFP4_MOE_OK"]) == L.OK
+    assert int(codes["MXFP4_MOE_ERR_INVALID_ARG"]) == L.ERR_INVALID_ARG
+    assert int(codes["MXFP4_MOE_ERR_WORKSPACE_TOO_SMALL"]) == L.ERR_WORKSPACE_TOO_SMALL
+    assert int(codes["MXFP4_MOE_ERR_UNSUPPORTED_DEVICE"]) == L.ERR_UNSUPPORTED_DEVICE
+    assert int(codes["MXFP4_MOE_ERR_CUDA"]) == L.ERR_CUDA
+    assert int(codes["MXFP4_MOE_ERR_DEVICE_TIMEOUT"]) == L.ERR_DEVICE_TIMEOUT
+    assert int(codes["MXFP4_MOE_ERR_DEVICE_BOUNDS"]) == L.ERR_DEVICE_BOUNDS
+    for c in (0, -1, -2, -3, -4, -5, -6, -99):
+        assert L.strerror(c)
+
+
+def _ws(L, *dims):
+    n = ctypes.c_size_t()
+    rc = L.lib.mxfp4_moe_workspace_size(ctypes.byref(L.Dims(*dims)), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_formula(L):
+    T, H, I, E, k = 8192, 2880, 2880, 32, 4
+    rc, n = _ws(L, T, H, I, E, k, 1.702, 7.0)
+    assert rc == 0
+    A = T * k
+    # saved h + act/dH + gathered rows dominate
+    assert n >= 2 * A * 2 * I * 2 + 2 * A * H + 4 * A * (I // 32)
+    assert n < 2 * A * 2 * I * 2 + 2 * A * H + 4 * A * (I // 32) + 4 * 1024 * 1024
+
+
+@pytest.mark.parametrize("dims", [
+    (0, 256, 256, 8, 2), (64, 250, 256, 8, 2), (64, 256, 100, 8, 2), (64, 256, 256, 0, 1),
+    (64, 256, 256, 8, 9), (64, 256, 256, 257, 2), (64, 256, 256, 8, 0),
+    (64, 256, 65536, 8, 2),  # tile scales would not fit shared memory
+])
+def test_bad_shapes_rejected(L, dims):
+    rc, _ = _ws(L, *dims, 1.702, 7.0)
+    assert rc == L.ERR_INVALID_ARG
+
+
+def test_null_pointers_rejected_before_device(L):
+    d = L.Dims(64, 256, 256, 8, 2, 1.702, 7.0)
+    w = L.Weights()
+    rc = L.lib.mxfp4_moe_forward(ctypes.byref(d), ctypes.byref(w), None, None, None, None, None,
+                                 None, 0, None)
+    assert rc == L.ERR_INVALID_ARG
+    rc = L.lib.mxfp4_moe_backward_input(ctypes.byref(d), ctypes.byref(w), None, 0, None, None, 0,
+                                        None, None, None, None)
+    assert rc == L.ERR_INVALID_ARG
+    rc = L.lib.mxfp4_moe_dequantize(None, None, 4, 64, None, None)
+    assert rc == L.ERR_INVALID_ARG
+    rc = L.lib.mxfp4_moe_dequantize(ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 48,
+                                    ctypes.c_void_p(16), None)
+    assert rc == L.ERR_INVALID_ARG  # K not a multiple of 32
+
+
+def test_small_workspace_rejected_before_device(L):
+    d = L.Dims(64, 256, 256, 8, 2, 1.702, 7.0)
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
+    w = L.Weights(p, p, p, p, p, p)
+    rc, need = _ws(L, 64, 256, 256, 8, 2, 1.702, 7.0)
+    rc = L.lib.mxfp4_moe_forward(ctypes.byref(d), ctypes.byref(w), p, p, p, None, None, p,
+                                 need - 1, None)
+    assert rc == L.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_python_wrappers_have_no_cpu_path():
+    """The torch-facing wrappers must refuse CPU tensors rather than compute on the host."""
+    import torch
+    from mxfp4_quantized_moe_b200 import moe
+    with pytest.raises(ValueError):
+        moe.dequantize(torch.zeros(4, 16, dtype=torch.uint8), torch.zeros(4, 1, dtype=torch.uint8))

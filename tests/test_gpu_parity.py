@@ -1,0 +1,201 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Bar: dequantized weights and top-k indices bit-exact; y, dX, d(routing weights) and
+d(logits) within max|err| <= 2e-2 * max|ref| per tensor with cosine >= 0.9999.
+The oracle and the CUDA path consume the same seeded inputs (the same fp32 logits), so
+routing must agree exactly.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from mxfp4_quantized_moe_b200 import inputs
+from oracle import mxfp4_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 2e-2
+COS_TOL = 0.9999
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from mxfp4_quantized_moe_b200 import moe as m
+    return m
+
+
+def assert_close(got, ref, name):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, name
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    err = float(np.max(np.abs(got - ref)))
+    scale = float(np.max(np.abs(ref)))
+    cos = float((got * ref).sum() / (np.linalg.norm(got) * np.linalg.norm(ref) + 1e-300))
+    assert err <= REL_TOL * scale, f"{name}: max|err| {err:.3e} > {REL_TOL} * {scale:.3e}"
+    assert cos >= COS_TOL, f"{name}: cosine {cos:.7f}"
+
+
+def run_block(moe, T, H, I, E, k, seed, tokens=None, **kw):
+    inp = inputs.make_layer(T, H, I, E, k, seed, **kw)
+    shape = moe.MoeShape(T, H, I, E, k)
+    w = moe.weights_to(inp, "cuda")
+    x, lg, dy = inp["x"].cuda(), inp["logits"].cuda(), inp["dy"].cuda()
+    ws = moe.alloc_workspace(shape)
+    wt = moe.transpose_weights(shape, w)
+    ti = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    y = moe.forward(shape, w, x, lg, ws, topk_idx=ti, topk_w=tw)
+    dx, dtw, dl = moe.backward_input(shape, w, wt, dy, ws)
+    rc, where = moe.device_check(ws)
+    assert rc == 0, f"device error {rc} at {where:#x}"
+    sel = np.arange(T) if tokens is None else np.asarray(tokens)
+    n = inputs.as_numpy(inp, sel)
+    f = O.moe_forward(n["x"], n["logits"], n["W"], k)
+    dX, dW, dL = O.moe_backward(n["dy"], f, n["W"])
+    got = {
+        "idx": ti.cpu().numpy()[sel], "w": tw.cpu().numpy()[sel], "y": y.float().cpu().numpy()[sel],
+        "dx": dx.float().cpu().numpy()[sel], "d_w": dtw.cpu().numpy()[sel],
+        "d_logits": dl.cpu().numpy()[sel],
+    }
+    ref = {"idx": f["idx"], "w": f["w"], "y": f["out"], "dx": dX, "d_w": dW, "d_logits": dL}
+    return got, ref
+
+
+def check_all(got, ref):
+    assert np.array_equal(got["idx"], ref["idx"]), "top-k indices differ"
+    np.testing.assert_allclose(got["w"], ref["w"], rtol=2e-6, atol=1e-7)
+    for name in ("y", "dx", "d_w", "d_logits"):
+        assert_close(got[name], ref[name], name)
+
+
+# ------------------------------------------------------------------ dequant -----------
+def test_dequant_bit_exact_all_codes_and_scales(moe):
+    rng = np.random.default_rng(0)
+    codes = np.arange(16)
+    s = np.arange(256)
+    cc, ss = np.meshgrid(codes, s, indexing="ij")
+    blocks = rng.integers(0, 256, (16 * 256, 32), dtype=np.uint8)
+    blocks[:, 0] = cc.ravel() | (np.roll(cc.ravel(), 5) << 4)
+    scales = np.stack([ss.ravel(), rng.integers(0, 256, 16 * 256)], 1).astype(np.uint8)
+    out = moe.dequantize(torch.from_numpy(blocks).cuda(), torch.from_numpy(scales).cuda())
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref = O.f64_to_bf16_bits(O.dequantize(blocks, scales))
+    assert np.array_equal(got, ref)
+
+
+def test_dequant_gpt_oss_rows_bit_exact(moe):
+    inp = inputs.make_layer(4, 2880, 2880, 2, 1, seed=9)
+    b, s = inp["gu_blocks"][1], inp["gu_scales"][1]
+    out = moe.dequantize(b.cuda(), s.cuda())
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, O.f64_to_bf16_bits(O.dequantize(b.numpy(), s.numpy())))
+
+
+def test_transposed_weights_are_a_pure_transpose(moe):
+    T, H, I, E, k = 8, 96, 160, 3, 2
+    inp = inputs.make_layer(T, H, I, E, k, seed=2)
+    shape = moe.MoeShape(T, H, I, E, k)
+    w = moe.weights_to(inp, "cuda")
+    wt = moe.transpose_weights(shape, w).cpu().numpy()
+
+    def unpack(b):
+        return np.stack([b & 15, b >> 4], -1).reshape(*b.shape[:-1], b.shape[-1] * 2)
+
+    def region(off, n):
+        start = (off + 255) // 256 * 256
+        return wt[start:start + n], start + n
+
+    o = 0
+    dn_t, o = region(o, E * I * H // 2)
+    gu_t, o = region(o, E * H * I)
+    dn_s, o = region(o, E * (I // 32) * H)
+    gu_s, o = region(o, E * (H // 32) * 2 * I)
+    dn = unpack(inp["dn_blocks"].numpy())  # [E][H][I]
+    gu = unpack(inp["gu_blocks"].numpy())  # [E][2I][H]
+    assert np.array_equal(unpack(dn_t.reshape(E, I, H // 2)), dn.transpose(0, 2, 1))
+    assert np.array_equal(unpack(gu_t.reshape(E, H, I)), gu.transpose(0, 2, 1))
+    assert np.array_equal(dn_s.reshape(E, I // 32, H), inp["dn_scales"].numpy().transpose(0, 2, 1))
+    assert np.array_equal(gu_s.reshape(E, H // 32, 2 * I), inp["gu_scales"].numpy().transpose(0, 2, 1))
+
+
+# ------------------------------------------------------------------ routing -----------
+def test_router_ties_and_topk_exact(moe):
+    T, H, I, E, k = 96, 64, 64, 8, 3
+    inp = inputs.make_layer(T, H, I, E, k, seed=3)
+    lg = inp["logits"].clone()
+    lg[0] = 1.0  # all equal: experts 0, 1, 2
+    lg[1, 5] = lg[1, 2] = lg[1].max() + 1  # tie at the top: 2 before 5
+    lg[2] = torch.arange(E, dtype=torch.float32)  # strictly increasing: 7, 6, 5
+    shape = moe.MoeShape(T, H, I, E, k)
+    w = moe.weights_to(inp, "cuda")
+    ws = moe.alloc_workspace(shape)
+    ti = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    moe.forward(shape, w, inp["x"].cuda(), lg.cuda(), ws, topk_idx=ti, topk_w=tw)
+    idx, wr = O.route(lg.numpy(), k)
+    got = ti.cpu().numpy()
+    assert got[0].tolist() == [0, 1, 2] and got[1, :2].tolist() == [2, 5]
+    assert got[2].tolist() == [7, 6, 5]
+    assert np.array_equal(got, idx)
+    np.testing.assert_allclose(tw.cpu().numpy(), wr, rtol=2e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------------ whole block -------
+def test_tiny_workload_full_parity(moe):
+    wl = inputs.WORKLOADS["tiny-moe-T64-H256-E8-k2"]
+    got, ref = run_block(moe, wl.T, wl.H, wl.I, wl.E, wl.k, seed=0)
+    check_all(got, ref)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,seed,kw", [
+    (1, 64, 64, 4, 2, 1, {}),                                  # a single token
+    (37, 96, 160, 5, 3, 4, {}),                                # K tails (96, 160, 320), ragged tiles
+    (5, 64, 64, 16, 1, 5, {}),                                 # most experts empty
+    (200, 128, 64, 4, 4, 6, {"scale_lo": 110, "scale_hi": 140}),  # k == E; scales above 2^1
+    (450, 64, 96, 2, 1, 7, {}),                                # several token tiles per expert
+    (130, 2880, 2880, 4, 2, 8, {}),                            # gpt-oss widths, few tokens
+])
+def test_edge_cases(moe, T, H, I, E, k, seed, kw):
+    got, ref = run_block(moe, T, H, I, E, k, seed, **kw)
+    check_all(got, ref)
+
+
+def test_expert_gradient_is_not_silent(moe):
+    """The pages' silent-gradient trap: dX must carry the expert path (not be zero)."""
+    got, ref = run_block(moe, 16, 64, 64, 4, 2, seed=12)
+    assert np.abs(got["dx"]).max() > 0.1 * np.abs(ref["dx"]).max() > 0
+    check_all(got, ref)
+
+
+def test_gpt_oss_20b_full_size_sampled_tokens(moe):
+    """The benchmarked launch configuration (T=8192, H=I=2880, E=32, k=4), checked on a seeded
+    sample of tokens: every token is independent, so the oracle runs on the sample only."""
+    wl = inputs.WORKLOADS["gpt-oss-20b-moe-T8192"]
+    sel = np.sort(np.random.default_rng(0).choice(wl.T, 48, replace=False))
+    got, ref = run_block(moe, wl.T, wl.H, wl.I, wl.E, wl.k, seed=0, tokens=sel)
+    check_all(got, ref)
+
+
+def test_zipf_skew_sampled_tokens(moe):
+    """Skewed routing (hottest expert ~25% of assignments, several experts under 16 rows)."""
+    sel = np.sort(np.random.default_rng(1).choice(4096, 32, replace=False))
+    got, ref = run_block(moe, 4096, 2880, 2880, 32, 4, seed=0, tokens=sel, zipf_s=1.2)
+    check_all(got, ref)
+
+
+def test_run_to_run_deterministic(moe):
+    T, H, I, E, k = 300, 256, 256, 8, 2
+    inp = inputs.make_layer(T, H, I, E, k, 13)
+    shape = moe.MoeShape(T, H, I, E, k)
+    w = moe.weights_to(inp, "cuda")
+    wt = moe.transpose_weights(shape, w)
+    outs = []
+    for _ in range(2):
+        ws = moe.alloc_workspace(shape)
+        y = moe.forward(shape, w, inp["x"].cuda(), inp["logits"].cuda(), ws)
+        dx, dtw, dl = moe.backward_input(shape, w, wt, inp["dy"].cuda(), ws)
+        outs.append([t.clone() for t in (y, dx, dtw, dl)])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)

@@ -153,6 +153,21 @@ def test_glu_backward_matches_finite_differences():
         assert fd == pytest.approx(dh[i], rel=1e-6, abs=1e-9)
 
 
+def test_clamp_masks_are_decided_on_bf16_preactivations():
+    # 7.01 rounds to bf16 7.0 (spacing 1/32 in [4, 8)): the gate clamp passes the gradient;
+    # 7.02 rounds to 7.03125 and blocks it.  Same for u at -7.01 / -7.02.
+    h = np.array([7.01, 1.0, 7.02, 1.0, 1.0, -7.01, 1.0, -7.02])
+    dact = np.ones(4)
+    hb = O.round_bf16(h)
+    assert hb.tolist() == [7.0, 1.0, 7.03125, 1.0, 1.0, -7.0, 1.0, -7.03125]
+    dh = O.glu_backward(h, dact, h_mask=hb)
+    assert dh[0] != 0 and dh[2] == 0 and dh[5] != 0 and dh[7] == 0
+    dh64 = O.glu_backward(h, dact)
+    assert dh64[0] == 0 and dh64[5] == 0
+    # away from the clamp the mask precision is irrelevant
+    assert dh[1] == dh64[1] and dh[4] == dh64[4]
+
+
 # ---------------------------------------------------------------- block -------------
 def test_scalar_twin_matches_oracle_brute_force():
     inp, n = _tiny()
@@ -336,6 +351,7 @@ def test_pins_catch_planted_mistakes(monkeypatch, mistake):
         monkeypatch.setattr(O, "_sigmoid", lambda z: 1.0 / (1.0 + np.exp(z)))
     elif mistake == "wrong_dact":
         orig_b = O.glu_backward
-        monkeypatch.setattr(O, "glu_backward", lambda h, d, a=1.702, l=7.0: orig_b(h, d, a, l)[..., ::-1])
+        monkeypatch.setattr(O, "glu_backward",
+                            lambda h, d, a=1.702, l=7.0, **kw: orig_b(h, d, a, l, **kw)[..., ::-1])
     with pytest.raises(AssertionError):
         _check_all_pins()
