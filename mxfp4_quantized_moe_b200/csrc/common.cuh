@@ -54,14 +54,19 @@ MOE_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
+// Suspend bound handed to mbarrier.try_wait (ns): a waiting thread sleeps until the phase
+// completes or this much time passes, so waiting warps do not take issue slots from the
+// warps that compute.
+constexpr uint32_t kSuspendHintNs = 200000;
+
 MOE_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -72,15 +77,13 @@ MOE_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const DevErr& err, int whe
                        volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
-      if (abort && *abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        err.set(MXFP4_MOE_ERR_DEVICE_TIMEOUT, where);
-        if (abort) *abort = 1;
-        return false;
-      }
+    if (abort && *abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      err.set(MXFP4_MOE_ERR_DEVICE_TIMEOUT, where);
+      if (abort) *abort = 1;
+      return false;
     }
   }
 }
@@ -204,6 +207,7 @@ MOE_DEV float bf16_to_f(uint16_t v) { return __uint_as_float((uint32_t)v << 16);
 MOE_DEV uint16_t f_to_bf16(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
+MOE_DEV float fast_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 MOE_DEV uint32_t pack_bf16x2(float lo, float hi) {
   return (uint32_t)f_to_bf16(lo) | ((uint32_t)f_to_bf16(hi) << 16);
 }

@@ -12,11 +12,16 @@
 // (A-from-TMEM form).  Shared memory carries only the token tile (TMA, 128B swizzle, B
 // operand) and the packed bytes, so its bandwidth goes to the MMA, not to the converter.
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: token tile + packed weight tile per k-step, scales per tile
+// Warp roles (512 threads, registers rebalanced per warpgroup with setmaxnreg):
+//   warp 0      TMA producer of the token ring (released by the MMA)
 //   warp 1      TMEM allocator and MMA issuer (one thread)
-//   warps 2-5   converters: packed MXFP4 -> bf16 -> TMEM (one TMEM lane quarter each)
-//   warps 6-9   epilogue: TMEM -> registers -> fused bias / GLU / routing / scatter
+//   warp 2      TMA producer of the packed-weight ring (released by the converters) and of
+//               the per-tile scales
+//   warps 4-11  converters: packed MXFP4 -> bf16 -> TMEM; two warps per TMEM lane quarter,
+//               taking alternate k-steps
+//   warps 12-15 epilogue: TMEM -> registers -> fused bias / GLU / routing / scatter
+// The token and weight rings are separate so that the converters can run ahead of the MMA
+// by the depth of the TMEM A ring without pinning token stages.
 // TMEM (512 columns): two fp32 accumulators of kBN columns (double buffered across tiles)
 // and a 4-stage ring of A operands (32 columns = 64 bf16 of K each).
 //
@@ -40,22 +45,30 @@ namespace moe {
 
 namespace {
 
-constexpr int kStages = 4;        // token + packed-weight ring depth
-constexpr int kAStages = 4;       // TMEM A ring depth
-constexpr int kThreads = 320;
+constexpr int kTStages = 5;       // token ring depth
+constexpr int kWStages = 8;       // packed-weight ring depth (even: a stage keeps its parity)
+constexpr int kAStages = 4;       // TMEM A ring depth (even, same reason)
+constexpr int kThreads = 512;
+constexpr int kConvWarps = 8;
 constexpr int kTokBytes = kBN * kBK * 2;      // 24 KB
 constexpr int kWBytes = kBM * (kBK / 2);      // 4 KB of packed nibbles
 constexpr int kAccCols = kBN;                 // fp32 accumulator columns per buffer
 constexpr int kACol0 = 2 * kAccCols;          // first TMEM column of the A ring
 constexpr int kTmemCols = 512;
+// registers per thread by warpgroup: control (producers, MMA), converters, epilogue
+constexpr int kRegsCtl = 56, kRegsConv = 128, kRegsEpi = 200;
+static_assert(128 * kRegsCtl + 256 * kRegsConv + 128 * kRegsEpi <= 65536, "register split");
 static_assert(kACol0 + kAStages * (kBK / 2) <= kTmemCols, "TMEM budget");
 static_assert(kBN % 32 == 0 && kBN <= 256, "token tile");
+static_assert(kWStages % 2 == 0 && kAStages % 2 == 0, "ring depths must be even");
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 struct __align__(8) Barriers {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t t_full[kTStages];
+  uint64_t t_empty[kTStages];
+  uint64_t w_full[kWStages];
+  uint64_t w_empty[kWStages];
   uint64_t a_full[kAStages];
   uint64_t a_empty[kAStages];
   uint64_t acc_full[2];
@@ -64,17 +77,24 @@ struct __align__(8) Barriers {
   uint64_t sc_empty[2];
   uint64_t drain;
 };
+static_assert(sizeof(Barriers) <= 512, "barrier block");
 
 struct SmemLayout {
   // offsets from the 1024-aligned dynamic smem base
-  static constexpr int tok = 0;
-  static constexpr int w = tok + kStages * kTokBytes;
-  static constexpr int bars = w + kStages * kWBytes;
-  static constexpr int misc = bars + 256;  // tmem slot, abort flag
-  static constexpr int cw = misc + 64;     // per converter warp: 2 x 2 x 32 scale words
-  static constexpr int tables = cw + 4 * 2 * 2 * 32 * 4;  // off[257], tile_start[257]
+  static constexpr int tok = 0;                                  // 1024-aligned (128B swizzle)
+  static constexpr int w = tok + kTStages * kTokBytes;           // 256-aligned (32B swizzle)
+  static constexpr int bars = w + kWStages * kWBytes;
+  static constexpr int misc = bars + 512;                        // tmem slot, abort flag
+  static constexpr int cw = misc + 64;                           // 8 warps x 2 x 32 scale words
+  static constexpr int tables = cw + kConvWarps * 2 * 32 * 4;    // off[257], tile_start[257]
   static constexpr int sc = ((tables + 2 * 257 * 4) + 127) / 128 * 128;  // 2 scale buffers
 };
+static_assert(SmemLayout::w % 1024 == 0, "weight ring alignment");
+
+template <uint32_t N>
+MOE_DEV void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <uint32_t N>
+MOE_DEV void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
 struct Tile {
   int e, fb, row0, n_valid, feat0;
@@ -82,13 +102,11 @@ struct Tile {
 
 __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const int* s_off, int E,
                                             int nfb, Tile& o) {
-  int lo = 0, hi = E;  // s_tstart[lo] <= t < s_tstart[hi]
+  int lo = 0, hi = E;  // largest lo with s_tstart[lo] <= t (s_tstart[E] = total > t)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (s_tstart[mid] <= t) lo = mid; else hi = mid;
   }
-  // skip experts with no tiles (equal starts)
-  while (lo + 1 <= E && s_tstart[lo + 1] <= t) ++lo;
   const int local = t - s_tstart[lo];
   const int tt = local / nfb;
   o.e = lo;
@@ -97,8 +115,6 @@ __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const in
   o.n_valid = min(kBN, s_off[lo + 1] - o.row0);
   o.feat0 = o.fb * kBM;
 }
-
-__device__ __forceinline__ float sigmoidf_fast(float z) { return 1.f / (1.f + __expf(-z)); }
 
 // In-register transpose-reduction: on entry v[c] is this lane's term for column c; on
 // exit v[0] holds, in lane l, the sum over the 32 lanes of the terms for column l.
@@ -114,6 +130,16 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane)
     }
   }
   return v[0];
+}
+
+// Last-phase parity of a ring stage after `issued` uses in total (for the exit drains).
+MOE_DEV bool drain_ring(uint64_t* full, int stages, int issued, const DevErr& err, int where) {
+  bool ok = true;
+  for (int s = 0; s < stages && s < issued; ++s) {
+    const int last = s + stages * ((issued - 1 - s) / stages);
+    ok &= mbar_wait(smem_u32(&full[s]), (last / stages) & 1, err, where, nullptr);
+  }
+  return ok;
 }
 
 template <int EPI, bool COLT>
@@ -143,9 +169,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     *s_abort = 0;
     mbar_init(smem_u32(&bar->drain), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&bar->full[s]), 1);
-      mbar_init(smem_u32(&bar->empty[s]), 1 + 4);  // MMA commit + 4 converter warps
+    for (int s = 0; s < kTStages; ++s) {
+      mbar_init(smem_u32(&bar->t_full[s]), 1);
+      mbar_init(smem_u32(&bar->t_empty[s]), 1);  // MMA commit
+    }
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(smem_u32(&bar->w_full[s]), 1);
+      mbar_init(smem_u32(&bar->w_empty[s]), 4);  // the 4 converter warps of this parity
     }
     for (int s = 0; s < kAStages; ++s) {
       mbar_init(smem_u32(&bar->a_full[s]), 4);
@@ -155,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bar->acc_full[s]), 1);
       mbar_init(smem_u32(&bar->acc_empty[s]), 4);
       mbar_init(smem_u32(&bar->sc_full[s]), 1);
-      mbar_init(smem_u32(&bar->sc_empty[s]), 4);
+      mbar_init(smem_u32(&bar->sc_empty[s]), kConvWarps);
     }
     fence_barrier_init();
   }
@@ -178,110 +208,133 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const int total = s_tstart[E];
+  const int wg = warp >> 2;
 
-  if (warp == 0) {
-    // ================================ TMA producer ==================================
-    int issued = 0, sc_issued = 0;
-    if (lane == 0) {
-      prefetch_tmap(&tmap_tok);
-      prefetch_tmap(&tmap_w);
-      int s = 0;
-      uint32_t ph = 0;
-      int lt = 0;
-      for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
-        Tile tl;
-        decode_tile(t, s_tstart, s_off, E, nfb, tl);
-        const int rows = min(kBM, N - tl.feat0);
-        const int sb = lt & 1;
-        if (!mbar_wait(smem_u32(&bar->sc_empty[sb]), ((lt >> 1) & 1) ^ 1, err, 0x200, s_abort)) break;
-        uint32_t bytes;
-        const uint8_t* src;
-        if (COLT) {
-          bytes = (uint32_t)(rows / 32) * K;
-          src = p.scales + ((size_t)tl.e * (N / 32) + tl.feat0 / 32) * K;
-        } else {
-          bytes = (uint32_t)rows * kb32;
-          src = p.scales + ((size_t)tl.e * N + tl.feat0) * kb32;
-        }
-        mbar_arrive_expect_tx(smem_u32(&bar->sc_full[sb]), bytes);
-        bulk_load(smem_u32(s_sc + sb * sc_bytes), src, bytes, smem_u32(&bar->sc_full[sb]));
-        ++sc_issued;
+  if (wg == 0) {
+    setmaxnreg_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ============================ token producer ==================================
+      int issued = 0;
+      if (lane == 0) {
+        prefetch_tmap(&tmap_tok);
         bool ok = true;
-        for (int ks = 0; ks < nk; ++ks) {
-          if (!mbar_wait(smem_u32(&bar->empty[s]), ph ^ 1, err, 0x201, s_abort)) { ok = false; break; }
-          const uint32_t fb = smem_u32(&bar->full[s]);
-          mbar_arrive_expect_tx(fb, kTokBytes + kWBytes);
-          tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
-                      tl.row0, fb);
-          tma_load_2d(smem_u32(smem + SmemLayout::w + s * kWBytes), &tmap_w, ks * (kBK / 2),
-                      tl.e * N + tl.feat0, fb);
-          ++issued;
-          if (++s == kStages) { s = 0; ph ^= 1; }
-        }
-        if (!ok) break;
-      }
-    }
-    __syncwarp();
-    // Drain: wait until every copy issued into a stage has landed before the CTA exits.
-    __syncthreads();
-    if (lane == 0) {
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last = s + kStages * ((issued - 1 - s) / kStages);
-        mbar_wait(smem_u32(&bar->full[s]), (last / kStages) & 1, err, 0x2F0, nullptr);
-      }
-      for (int sb = 0; sb < 2 && sb < sc_issued; ++sb) {
-        const int last = sb + 2 * ((sc_issued - 1 - sb) / 2);
-        mbar_wait(smem_u32(&bar->sc_full[sb]), (last / 2) & 1, err, 0x2F1, nullptr);
-      }
-    }
-  } else if (warp == 1) {
-    // ================================ MMA issuer ====================================
-    if (lane == 0) {
-      int s = 0, sa = 0;
-      uint32_t ph = 0, aph = 0;
-      int lt = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
-        Tile tl;
-        decode_tile(t, s_tstart, s_off, E, nfb, tl);
-        const int acc = lt & 1;
-        if (!mbar_wait(smem_u32(&bar->acc_empty[acc]), ((lt >> 1) & 1) ^ 1, err, 0x300, s_abort)) break;
-        tc_fence_after();
-        const uint32_t idesc = idesc_bf16_m128((tl.n_valid + 15) & ~15);
-        const uint32_t d_tmem = tmem + acc * kAccCols;
-        for (int ks = 0; ks < nk; ++ks) {
-          if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort) ||
-              !mbar_wait(smem_u32(&bar->a_full[sa]), aph, err, 0x302, s_abort)) {
-            ok = false;
-            break;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+          Tile tl;
+          decode_tile(t, s_tstart, s_off, E, nfb, tl);
+          for (int ks = 0; ks < nk; ++ks) {
+            const int s = issued % kTStages;
+            if (!mbar_wait(smem_u32(&bar->t_empty[s]), ((issued / kTStages) & 1) ^ 1, err, 0x201,
+                           s_abort)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&bar->t_full[s]);
+            mbar_arrive_expect_tx(fb, kTokBytes);
+            tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
+                        tl.row0, fb);
+            ++issued;
           }
-          tc_fence_after();
-          const uint64_t bdesc =
-              smem_desc_kmajor_sw128(smem_u32(smem + SmemLayout::tok + s * kTokBytes));
-          const uint32_t a_tmem = tmem + kACol0 + sa * (kBK / 2);
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
-                        (ks | kk) != 0);
-          mma_commit(smem_u32(&bar->empty[s]));
-          mma_commit(smem_u32(&bar->a_empty[sa]));
-          if (++s == kStages) { s = 0; ph ^= 1; }
-          if (++sa == kAStages) { sa = 0; aph ^= 1; }
         }
-        if (ok) mma_commit(smem_u32(&bar->acc_full[acc]));
       }
-      // every MMA issued by this thread has completed once `drain` flips
-      mma_commit(smem_u32(&bar->drain));
-      mbar_wait(smem_u32(&bar->drain), 0, err, 0x3F0, nullptr);
+      __syncwarp();
+      __syncthreads();
+      // exit drain: every token copy issued has landed
+      if (lane == 0) drain_ring(bar->t_full, kTStages, issued, err, 0x2F0);
+    } else if (warp == 2) {
+      // ============================ weight + scale producer =========================
+      int issued = 0, sc_issued = 0;
+      if (lane == 0) {
+        prefetch_tmap(&tmap_w);
+        bool ok = true;
+        int lt = 0;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+          Tile tl;
+          decode_tile(t, s_tstart, s_off, E, nfb, tl);
+          const int rows = min(kBM, N - tl.feat0);
+          const int sb = lt & 1;
+          if (!mbar_wait(smem_u32(&bar->sc_empty[sb]), ((lt >> 1) & 1) ^ 1, err, 0x200, s_abort)) break;
+          uint32_t bytes;
+          const uint8_t* src;
+          if (COLT) {
+            bytes = (uint32_t)(rows / 32) * K;
+            src = p.scales + ((size_t)tl.e * (N / 32) + tl.feat0 / 32) * K;
+          } else {
+            bytes = (uint32_t)rows * kb32;
+            src = p.scales + ((size_t)tl.e * N + tl.feat0) * kb32;
+          }
+          mbar_arrive_expect_tx(smem_u32(&bar->sc_full[sb]), bytes);
+          bulk_load(smem_u32(s_sc + sb * sc_bytes), src, bytes, smem_u32(&bar->sc_full[sb]));
+          ++sc_issued;
+          for (int ks = 0; ks < nk; ++ks) {
+            const int s = issued % kWStages;
+            if (!mbar_wait(smem_u32(&bar->w_empty[s]), ((issued / kWStages) & 1) ^ 1, err, 0x202,
+                           s_abort)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&bar->w_full[s]);
+            mbar_arrive_expect_tx(fb, kWBytes);
+            tma_load_2d(smem_u32(smem + SmemLayout::w + s * kWBytes), &tmap_w, ks * (kBK / 2),
+                        tl.e * N + tl.feat0, fb);
+            ++issued;
+          }
+        }
+      }
+      __syncwarp();
+      __syncthreads();
+      if (lane == 0) {
+        drain_ring(bar->w_full, kWStages, issued, err, 0x2F1);
+        drain_ring(bar->sc_full, 2, sc_issued, err, 0x2F2);
+      }
+    } else if (warp == 1) {
+      // ============================ MMA issuer ======================================
+      if (lane == 0) {
+        int g = 0;  // k-steps issued so far (all tiles)
+        int lt = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+          Tile tl;
+          decode_tile(t, s_tstart, s_off, E, nfb, tl);
+          const int acc = lt & 1;
+          if (!mbar_wait(smem_u32(&bar->acc_empty[acc]), ((lt >> 1) & 1) ^ 1, err, 0x300, s_abort)) break;
+          tc_fence_after();
+          const uint32_t idesc = idesc_bf16_m128((tl.n_valid + 15) & ~15);
+          const uint32_t d_tmem = tmem + acc * kAccCols;
+          for (int ks = 0; ks < nk; ++ks, ++g) {
+            const int s = g % kTStages, sa = g % kAStages;
+            if (!mbar_wait(smem_u32(&bar->t_full[s]), (g / kTStages) & 1, err, 0x301, s_abort) ||
+                !mbar_wait(smem_u32(&bar->a_full[sa]), (g / kAStages) & 1, err, 0x302, s_abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t bdesc =
+                smem_desc_kmajor_sw128(smem_u32(smem + SmemLayout::tok + s * kTokBytes));
+            const uint32_t a_tmem = tmem + kACol0 + sa * (kBK / 2);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
+                          (ks | kk) != 0);
+            mma_commit(smem_u32(&bar->t_empty[s]));
+            mma_commit(smem_u32(&bar->a_empty[sa]));
+          }
+          if (ok) mma_commit(smem_u32(&bar->acc_full[acc]));
+        }
+        // every MMA issued by this thread has completed once `drain` flips
+        mma_commit(smem_u32(&bar->drain));
+        mbar_wait(smem_u32(&bar->drain), 0, err, 0x3F0, nullptr);
+      }
+      __syncwarp();
+      __syncthreads();
+    } else {
+      __syncthreads();
     }
-    __syncwarp();
-    __syncthreads();
-  } else if (warp < 6) {
+  } else if (wg < 3) {
     // ================================ converters ====================================
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint32_t* cw = reinterpret_cast<uint32_t*>(smem + SmemLayout::cw) + (warp - 2) * 128;
-    int s = 0, sa = 0;
-    uint32_t ph = 0, aph = 0;
+    // Converter warp c (0..7) serves TMEM lane quarter q = warp % 4 and the k-steps whose
+    // running index g has parity c / 4; its partner warp takes the other parity.
+    const int q = warp & 3;
+    const int cidx = warp - 4;
+    const int par = cidx >> 2;
+    uint32_t* cw = reinterpret_cast<uint32_t*>(smem + SmemLayout::cw) + cidx * 64;
+    const int r = 32 * q + lane;  // row of the 128-row weight tile
+    // 32B-swizzled packed tile: the two 16-byte halves of row r swap when bit 2 of r is set
+    const int swz = (r >> 2) & 1;
+    int g = 0;
     int lt = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
@@ -291,33 +344,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sb = lt & 1;
       if (!mbar_wait(smem_u32(&bar->sc_full[sb]), (lt >> 1) & 1, err, 0x400, s_abort)) break;
       const uint8_t* scb = s_sc + sb * sc_bytes;
-      const int r = 32 * q + lane;  // row of the 128-row weight tile
-      for (int ks = 0; ks < nk; ++ks) {
-        if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x401, s_abort)) { ok = false; break; }
+      for (int ks = 0; ks < nk; ++ks, ++g) {
+        if ((g & 1) != par) continue;
+        const int s = g % kWStages;
+        if (!mbar_wait(smem_u32(&bar->w_full[s]), (g / kWStages) & 1, err, 0x401, s_abort)) {
+          ok = false;
+          break;
+        }
         uint32_t qw[8];
         {
-          const uint4* wp =
-              reinterpret_cast<const uint4*>(smem + SmemLayout::w + s * kWBytes + r * (kBK / 2));
-          const uint4 w0 = wp[0], w1 = wp[1];
+          const uint8_t* row = smem + SmemLayout::w + s * kWBytes + r * (kBK / 2);
+          const uint4 w0 = *reinterpret_cast<const uint4*>(row + (swz << 4));
+          const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((swz ^ 1) << 4));
           qw[0] = w0.x; qw[1] = w0.y; qw[2] = w0.z; qw[3] = w0.w;
           qw[4] = w1.x; qw[5] = w1.y; qw[6] = w1.z; qw[7] = w1.w;
         }
         // scale factors: f1 (and f2 when some scale is above 128), as bf16x2 words
-        uint32_t f1a, f1b, f2a = 0x3F803F80u, f2b = 0x3F803F80u;
+        uint32_t f1a = 0, f1b = 0, f2a = 0x3F803F80u, f2b = 0x3F803F80u;
         bool slow;
         if (!COLT) {
-          const uint32_t sa_ = active ? scb[r * kb32 + 2 * ks] : 127u;
-          const uint32_t sb_ = (active && 2 * ks + 1 < kb32) ? scb[r * kb32 + 2 * ks + 1] : 127u;
-          f1a = dup16(ue8m0_f1(sa_));
-          f1b = dup16(ue8m0_f1(sb_));
-          slow = __any_sync(kFull, (sa_ > 128u) | (sb_ > 128u));
+          const uint32_t sA = active ? scb[r * kb32 + 2 * ks] : 127u;
+          const uint32_t sB = (active && 2 * ks + 1 < kb32) ? scb[r * kb32 + 2 * ks + 1] : 127u;
+          f1a = dup16(ue8m0_f1(sA));
+          f1b = dup16(ue8m0_f1(sB));
+          slow = __any_sync(kFull, (sA > 128u) | (sB > 128u));
           if (slow) {
-            f2a = dup16(ue8m0_f2(sa_));
-            f2b = dup16(ue8m0_f2(sb_));
+            f2a = dup16(ue8m0_f2(sA));
+            f2b = dup16(ue8m0_f2(sB));
           }
         } else {
-          // lane l computes the factors of K elements 2l, 2l+1 of this k-step; the
-          // warp shares them through shared memory (same scale row for all 32 lanes).
+          // lane l computes the factors of K elements 2l, 2l+1 of this k-step; the warp
+          // shares them through shared memory (one scale row for all 32 lanes).
           const int k0 = ks * kBK + 2 * lane;
           uint32_t s0 = 127u, s1 = 127u;
           if (active && k0 < K) {
@@ -325,14 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             s1 = (k0 + 1 < K) ? scb[q * K + k0 + 1] : 127u;
           }
           slow = __any_sync(kFull, (s0 > 128u) | (s1 > 128u));
-          uint32_t* cwb = cw + (ks & 1) * 64;
-          cwb[lane] = ue8m0_f1(s0) | (ue8m0_f1(s1) << 16);
-          if (slow) cwb[32 + lane] = ue8m0_f2(s0) | (ue8m0_f2(s1) << 16);
-          f1a = f1b = 0;
+          cw[lane] = ue8m0_f1(s0) | (ue8m0_f1(s1) << 16);
+          if (slow) cw[32 + lane] = ue8m0_f2(s0) | (ue8m0_f2(s1) << 16);
         }
-        // the packed bytes are in registers: release the stage's weight half
+        // the packed bytes are in registers: release the weight stage
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar->empty[s]));
+        if (lane == 0) mbar_arrive(smem_u32(&bar->w_empty[s]));
 
         uint32_t out[32];
         if (active) {
@@ -350,12 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int m = 0; m < 32; ++m) out[m] = bmul2(out[m], m < 16 ? f2a : f2b);
             }
           } else {
-            const uint32_t* cwb = cw + (ks & 1) * 64;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               uint32_t pt[4];
               e2m1x8_to_bf16x2_pattern(qw[i], pt);
-              const uint4 f = *reinterpret_cast<const uint4*>(cwb + 4 * i);
+              const uint4 f = *reinterpret_cast<const uint4*>(cw + 4 * i);
               out[4 * i + 0] = bmul2(pt[0], f.x);
               out[4 * i + 1] = bmul2(pt[1], f.y);
               out[4 * i + 2] = bmul2(pt[2], f.z);
@@ -364,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (slow) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const uint4 f = *reinterpret_cast<const uint4*>(cwb + 32 + 4 * i);
+                const uint4 f = *reinterpret_cast<const uint4*>(cw + 32 + 4 * i);
                 out[4 * i + 0] = bmul2(out[4 * i + 0], f.x);
                 out[4 * i + 1] = bmul2(out[4 * i + 1], f.y);
                 out[4 * i + 2] = bmul2(out[4 * i + 2], f.z);
@@ -373,18 +427,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (!mbar_wait(smem_u32(&bar->a_empty[sa]), aph ^ 1, err, 0x402, s_abort)) { ok = false; break; }
+        const int sa = g % kAStages;
+        if (!mbar_wait(smem_u32(&bar->a_empty[sa]), ((g / kAStages) & 1) ^ 1, err, 0x402,
+                       s_abort)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         if (active) {
           tmem_st32(tmem + ((uint32_t)(32 * q) << 16) + kACol0 + sa * (kBK / 2), out);
           tmem_wait_st();
         }
         tc_fence_before();
-        __syncwarp();
+        __syncwarp();  // also orders this k-step's reads of cw before the next writes
         if (lane == 0) mbar_arrive(smem_u32(&bar->a_full[sa]));
-        if (++s == kStages) { s = 0; ph ^= 1; }
-        if (++sa == kAStages) { sa = 0; aph ^= 1; }
       }
+      if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar->sc_empty[sb]));
     }
@@ -392,6 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   } else {
     // ================================ epilogue ======================================
+    setmaxnreg_inc<kRegsEpi>();
     const int q = warp & 3;
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
@@ -412,25 +471,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!active) continue;
         const int ncol = min(32, tl.n_valid - c0);
         const int rbase = tl.row0 + c0;
+        const bool odd = (lane & 1) != 0;
         if (EPI == kEpiGateUp) {
-          // h = acc + bias (interleaved: even f = gate, odd f = up); act from the pair
+          // Columns j (even lane) and j+1 (odd lane) of each pair: the lanes of an
+          // interleaved (gate, up) feature pair swap one value so that each holds (g, u) of
+          // its own column; it stores h as one bf16x2 word and act as one bf16.
           const int I = N >> 1;
-          const bool gate = (lane & 1) == 0;
           const int jf = f >> 1;
+          uint32_t hw[16];
+          float av[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float v0 = __uint_as_float(r[j]) + bias_f;
-            const float v1 = __uint_as_float(r[j + 1]) + bias_f;
-            if (j < ncol) p.out0[(size_t)(rbase + j) * N + f] = f_to_bf16(v0);
-            if (j + 1 < ncol) p.out0[(size_t)(rbase + j + 1) * N + f] = f_to_bf16(v1);
-            const float recv = __shfl_xor_sync(kFull, gate ? v1 : v0, 1);
-            const float g = gate ? v0 : recv;
-            const float u = gate ? recv : v1;
-            const int col = j + (gate ? 0 : 1);
+          for (int jj = 0; jj < 16; ++jj) {
+            const float v0 = __uint_as_float(r[2 * jj]) + bias_f;
+            const float v1 = __uint_as_float(r[2 * jj + 1]) + bias_f;
+            const float recv = __shfl_xor_sync(kFull, odd ? v0 : v1, 1);
+            const float g = odd ? recv : v0;
+            const float u = odd ? v1 : recv;
+            hw[jj] = pack_bf16x2(g, u);
             const float gc = fminf(g, p.limit);
             const float uc = fminf(fmaxf(u, -p.limit), p.limit);
-            const float a = (uc + 1.f) * gc * sigmoidf_fast(p.alpha * gc);
-            if (col < ncol) p.out1[(size_t)(rbase + col) * I + jf] = f_to_bf16(a);
+            av[jj] = (uc + 1.f) * gc * fast_sigmoid(p.alpha * gc);
+          }
+          uint32_t* hrow = reinterpret_cast<uint32_t*>(p.out0);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int col = 2 * jj + (odd ? 1 : 0);
+            if (col < ncol) {
+              hrow[((size_t)(rbase + col) * N + (f & ~1)) >> 1] = hw[jj];
+              p.out1[(size_t)(rbase + col) * I + jf] = f_to_bf16(av[jj]);
+            }
           }
         } else {
           int my_slot = 0;
@@ -440,38 +509,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (EPI == kEpiDown || EPI == kEpiDact) my_w = p.topk_w[my_slot];
           }
           if (EPI == kEpiDown || EPI == kEpiDx) {
+            // Feature pairs (f, f+1) live in lanes (2m, 2m+1): after one swap the even lane
+            // holds both features of column j, the odd lane both of column j+1.
+            uint32_t ow[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int slot = __shfl_sync(kFull, my_slot, j);
-              float v = __uint_as_float(r[j]);
-              if (EPI == kEpiDown) v = __shfl_sync(kFull, my_w, j) * (v + bias_f);
-              if (j < ncol) p.out0[(size_t)slot * N + f] = f_to_bf16(v);
+            for (int jj = 0; jj < 16; ++jj) {
+              float v0 = __uint_as_float(r[2 * jj]);
+              float v1 = __uint_as_float(r[2 * jj + 1]);
+              if (EPI == kEpiDown) {
+                v0 = __shfl_sync(kFull, my_w, 2 * jj) * (v0 + bias_f);
+                v1 = __shfl_sync(kFull, my_w, 2 * jj + 1) * (v1 + bias_f);
+              }
+              const float recv = __shfl_xor_sync(kFull, odd ? v0 : v1, 1);
+              ow[jj] = odd ? pack_bf16x2(recv, v1) : pack_bf16x2(v0, recv);
+            }
+            uint32_t* orow = reinterpret_cast<uint32_t*>(p.out0);
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int col = 2 * jj + (odd ? 1 : 0);
+              const int slot = __shfl_sync(kFull, my_slot, col);
+              if (col < ncol) orow[((size_t)slot * N + (f & ~1)) >> 1] = ow[jj];
             }
           } else {  // kEpiDact
             const int I = N;
-            float part[32];
             const uint32_t* hw = reinterpret_cast<const uint32_t*>(p.hsaved);
             uint32_t* dh = reinterpret_cast<uint32_t*>(p.out0);
+            // issue all 32 loads of the saved (g, u) pairs first (h is read-only here);
+            // columns past the tile's rows read a valid row and are discarded
+            uint32_t hv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int row = min(rbase + j, p.A - 1);
+              hv[j] = __ldg(hw + (size_t)row * I + f);
+            }
+            float part[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float wr = __shfl_sync(kFull, my_w, j);
-              part[j] = 0.f;
-              if (j < ncol) {
-                const uint32_t hv = hw[(size_t)(rbase + j) * I + f];
-                const float g = bf16_lo(hv), u = bf16_hi(hv);
-                const float dz = __uint_as_float(r[j]);
-                const float gc = fminf(g, p.limit);
-                const float uc = fminf(fmaxf(u, -p.limit), p.limit);
-                const float sg = sigmoidf_fast(p.alpha * gc);
-                part[j] = dz * ((uc + 1.f) * gc * sg);
-                const float dact = wr * dz;
-                const float dg = (g <= p.limit)
-                                     ? dact * (uc + 1.f) * (sg + p.alpha * gc * sg * (1.f - sg))
-                                     : 0.f;
-                const float du = (u >= -p.limit && u <= p.limit) ? dact * gc * sg : 0.f;
-                dh[(size_t)(rbase + j) * I + f] = pack_bf16x2(dg, du);
-              }
+              const float g = bf16_lo(hv[j]), u = bf16_hi(hv[j]);
+              const float dz = __uint_as_float(r[j]);
+              const float gc = fminf(g, p.limit);
+              const float uc = fminf(fmaxf(u, -p.limit), p.limit);
+              const float sg = fast_sigmoid(p.alpha * gc);
+              part[j] = (j < ncol) ? dz * ((uc + 1.f) * gc * sg) : 0.f;
+              const float dact = wr * dz;
+              const float dg = (g <= p.limit)
+                                   ? dact * (uc + 1.f) * (sg + p.alpha * gc * sg * (1.f - sg))
+                                   : 0.f;
+              const float du = (u >= -p.limit && u <= p.limit) ? dact * gc * sg : 0.f;
+              hv[j] = pack_bf16x2(dg, du);
             }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < ncol) dh[(size_t)(rbase + j) * I + f] = hv[j];
             const float sum = warp_transpose_reduce(part, lane);
             if (lane < ncol) p.dw_part[(size_t)((tl.feat0 >> 5) + q) * p.A + rbase + lane] = sum;
           }
@@ -550,7 +640,7 @@ cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const uint16_t*
     const cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)kBM};
     const cuuint32_t es[2] = {1, 1};
     if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(wq), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }

@@ -43,6 +43,8 @@ class Workload:
 WORKLOADS = {
     "tiny-moe-T64-H256-E8-k2": Workload("tiny-moe-T64-H256-E8-k2", 64, 256, 256, 8, 2),
     "gpt-oss-20b-moe-T8192": Workload("gpt-oss-20b-moe-T8192", 8192, 2880, 2880, 32, 4),
+    # smaller batch of the same layer, for profiler captures that must stay a few GB
+    "gpt-oss-20b-moe-T4096": Workload("gpt-oss-20b-moe-T4096", 4096, 2880, 2880, 32, 4),
     "gpt-oss-120b-moe-T16384": Workload("gpt-oss-120b-moe-T16384", 16384, 2880, 2880, 128, 4),
     "gpt-oss-20b-moe-zipf-T16384": Workload("gpt-oss-20b-moe-zipf-T16384", 16384, 2880, 2880, 32, 4,
                                             zipf_s=1.2),

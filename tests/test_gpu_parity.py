@@ -32,6 +32,9 @@ def assert_close(got, ref, name):
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
     err = float(np.max(np.abs(got - ref)))
     scale = float(np.max(np.abs(ref)))
+    if scale == 0.0:  # degenerate case (e.g. d_logits with k == 1): must be exactly zero
+        assert err == 0.0, f"{name}: expected all zeros, max|got| {err:.3e}"
+        return
     cos = float((got * ref).sum() / (np.linalg.norm(got) * np.linalg.norm(ref) + 1e-300))
     assert err <= REL_TOL * scale, f"{name}: max|err| {err:.3e} > {REL_TOL} * {scale:.3e}"
     assert cos >= COS_TOL, f"{name}: cosine {cos:.7f}"
