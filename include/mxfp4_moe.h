@@ -133,6 +133,33 @@ MXFP4_MOE_API int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_wei
                       const float* logits, uint16_t* y, int32_t* topk_idx, float* topk_w,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* Forward for callers that cannot allocate device memory (no counterpart in the source pages:
+ * a deployment form of mxfp4_moe_forward, not part of the method).
+ * Who needs it: code that runs the layer where it holds no device allocator -- an
+ * inference-engine plugin whose enqueue step receives only input and output pointers, a
+ * process whose device memory belongs to another framework's pool, or a latency-critical
+ * serving loop that cannot pay for cudaMalloc's implicit device synchronization.
+ * What it does: exactly mxfp4_moe_forward, with the workspace taken from a fixed array of
+ * MXFP4_MOE_STATIC_SCRATCH_BYTES (64 MiB) that the library holds in device memory on every
+ * GPU where this entry point has run (allocated when the library's code is loaded there, kept
+ * until the process exits).  Arguments mean what they mean for mxfp4_moe_forward; the caller
+ * still provides x, logits, y and the optional topk_idx / topk_w.  No cudaMalloc, cudaFree or
+ * other allocating call is made.
+ * First call on a device: it looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current and caches it, so make that first call before any stream capture.
+ * Sharing: every call uses the same array and leaves its contents there for the next call; the
+ * call clears what must start at zero.  Calls that overlap on the GPU (other streams, other
+ * host threads) race on the array and must be serialized by the caller.  The saved state it
+ * leaves is not usable by mxfp4_moe_backward_input, and device-side faults of this form are
+ * not reported (use the workspace form and mxfp4_moe_check to diagnose).
+ * Errors: WORKSPACE_TOO_SMALL when mxfp4_moe_workspace_size(d) exceeds
+ * MXFP4_MOE_STATIC_SCRATCH_BYTES (at H = I = 2880, k = 4 that is above about 575 tokens);
+ * otherwise as mxfp4_moe_forward. */
+#define MXFP4_MOE_STATIC_SCRATCH_BYTES (64ull << 20)
+MXFP4_MOE_API int mxfp4_moe_forward_static(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w,
+                                           const uint16_t* x, const float* logits, uint16_t* y,
+                                           int32_t* topk_idx, float* topk_w, void* stream);
+
 /* Input-gradient backward through the frozen quantized weights (no weight gradient).
  *   wt       the transposed copy from mxfp4_moe_transpose_weights for the same weights
  *   dy       bf16 [T][H]  upstream gradient dL/d(out)

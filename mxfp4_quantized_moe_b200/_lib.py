@@ -49,6 +49,8 @@ SIGNATURES = {
                                                    _vp, _sz, _vp]),
     "mxfp4_moe_forward": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Weights), _vp, _vp,
                                          _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mxfp4_moe_forward_static": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Weights),
+                                                _vp, _vp, _vp, _vp, _vp, _vp]),
     "mxfp4_moe_backward_input": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Weights),
                                                 _vp, _sz, _vp, _vp, _sz, _vp, _vp, _vp, _vp]),
     "mxfp4_moe_dequantize": (ctypes.c_int, [_vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp]),
