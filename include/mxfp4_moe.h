@@ -98,8 +98,9 @@ typedef struct {
 } mxfp4_moe_weights;
 
 /* Bytes of device workspace that mxfp4_moe_forward / mxfp4_moe_backward_input need for `d`.
- * The forward leaves its saved state (routing, permutation, gate_up pre-activations) in the
- * workspace; the backward reads it and uses the rest as scratch.
+ * The forward leaves its saved state in the workspace (routing, permutation, the GLU output and
+ * its two derivative factors per (assignment, feature)); the backward reads it and uses the
+ * rest as scratch.
  * Errors: INVALID_ARG (null pointers, bad shape). */
 MXFP4_MOE_API int mxfp4_moe_workspace_size(const mxfp4_moe_dims* d, size_t* bytes);
 
@@ -153,7 +154,7 @@ MXFP4_MOE_API int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_wei
  * leaves is not usable by mxfp4_moe_backward_input, and device-side faults of this form are
  * not reported (use the workspace form and mxfp4_moe_check to diagnose).
  * Errors: WORKSPACE_TOO_SMALL when mxfp4_moe_workspace_size(d) exceeds
- * MXFP4_MOE_STATIC_SCRATCH_BYTES (at H = I = 2880, k = 4 that is above about 575 tokens);
+ * MXFP4_MOE_STATIC_SCRATCH_BYTES (at H = I = 2880, k = 4 that is above 480 tokens);
  * otherwise as mxfp4_moe_forward. */
 #define MXFP4_MOE_STATIC_SCRATCH_BYTES (64ull << 20)
 MXFP4_MOE_API int mxfp4_moe_forward_static(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w,

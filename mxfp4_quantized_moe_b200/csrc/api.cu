@@ -13,7 +13,7 @@ constexpr size_t kAlign = 256;
 size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-  size_t err, hist, off, idx, w, perm, inv, h, act_dh, rows, cbias, dwp, total;
+  size_t err, hist, off, idx, w, perm, inv, dgu, act, dh, rows, cbias, dwp, dw, total;
 };
 
 WsLayout ws_layout(const mxfp4_moe_dims& d) {
@@ -27,11 +27,13 @@ WsLayout ws_layout(const mxfp4_moe_dims& d) {
   L.w = o;      o = up(o + 4 * A);
   L.perm = o;   o = up(o + 4 * A);
   L.inv = o;    o = up(o + 4 * A);
-  L.h = o;      o = up(o + 2 * A * 2 * d.I);   // saved gate_up pre-activations
-  L.act_dh = o; o = up(o + 2 * A * 2 * d.I);   // act [A][I] (fwd) / dH [A][2I] (bwd)
+  L.dgu = o;    o = up(o + 4 * A * d.I);       // saved GLU derivative factors (bf16 pairs)
+  L.act = o;    o = up(o + 2 * A * d.I);       // saved act [A][I]
+  L.dh = o;     o = up(o + 2 * A * 2 * d.I);   // dH [A][2I] (backward scratch)
   L.rows = o;   o = up(o + 2 * A * d.H);       // Xp/Yslot (fwd), dYp/dXslot (bwd)
   L.cbias = o;  o = up(o + 4 * A);
   L.dwp = o;    o = up(o + 4 * A * (d.I / 32));
+  L.dw = o;     o = up(o + 4 * A);
   L.total = o;
   return L;
 }
@@ -213,8 +215,8 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
   float* wr = at<float>(ws, L.w);
   int32_t* perm = at<int32_t>(ws, L.perm);
   int32_t* inv = at<int32_t>(ws, L.inv);
-  uint16_t* h = at<uint16_t>(ws, L.h);
-  uint16_t* act = at<uint16_t>(ws, L.act_dh);
+  uint16_t* dgu = at<uint16_t>(ws, L.dgu);
+  uint16_t* act = at<uint16_t>(ws, L.act);
   uint16_t* rows = at<uint16_t>(ws, L.rows);
 
   MOE_TRY(cudaMemsetAsync(hist, 0, 4ull * E, st));
@@ -225,8 +227,8 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
   moe::GemmArgs g{};
   g.off = off; g.E = E; g.A = A; g.perm = perm; g.topk_w = wr; g.err = err;
   g.alpha = d->glu_alpha; g.limit = d->glu_limit;
-  // gate_up: h = Xp W_gu^T + b_gu, act = GLU(h)
-  g.scales = w->gu_scales; g.K = H; g.N = 2 * I; g.bias = w->gu_bias; g.out0 = h; g.out1 = act;
+  // gate_up: h = Xp W_gu^T + b_gu; act = GLU(h) and the GLU derivative factors are saved
+  g.scales = w->gu_scales; g.K = H; g.N = 2 * I; g.bias = w->gu_bias; g.out0 = dgu; g.out1 = act;
   MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, rows, w->gu_blocks, g, sms, st));
   // down: Yslot[slot] = w_slot * (act W_d^T + b_d)
   g.scales = w->dn_scales; g.K = I; g.N = H; g.bias = w->dn_bias; g.out0 = rows; g.out1 = nullptr;
@@ -260,9 +262,10 @@ int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* wr = at<float>(ws, L.w);
   int32_t* perm = at<int32_t>(ws, L.perm);
-  int32_t* inv = at<int32_t>(ws, L.inv);
-  uint16_t* h = at<uint16_t>(ws, L.h);
-  uint16_t* dh = at<uint16_t>(ws, L.act_dh);
+  const uint32_t* dgu = at<uint32_t>(ws, L.dgu);
+  const uint16_t* act = at<uint16_t>(ws, L.act);
+  uint16_t* dh = at<uint16_t>(ws, L.dh);
+  float* dw = at<float>(ws, L.dw);
   uint16_t* rows = at<uint16_t>(ws, L.rows);
   float* cbias = at<float>(ws, L.cbias);
   float* dwp = at<float>(ws, L.dwp);
@@ -273,15 +276,16 @@ int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w
   g.off = off; g.E = E; g.A = A; g.perm = perm; g.topk_w = wr; g.err = err;
   g.alpha = d->glu_alpha; g.limit = d->glu_limit;
   // dZ = dYp W_d (contract over H); epilogue: GLU derivative -> dH, partial <dZ, act>
-  g.scales = at<uint8_t>(wtp, LT.dn_scales); g.K = H; g.N = I; g.out0 = dh; g.hsaved = h;
+  g.scales = at<uint8_t>(wtp, LT.dn_scales); g.K = H; g.N = I; g.out0 = dh; g.dgu = dgu; g.act = act;
   g.dw_part = dwp;
   MOE_LAUNCH("gemm_dact_glu_bwd", moe::launch_grouped_gemm(moe::kEpiDact, true, rows, at<uint8_t>(wtp, LT.dn_blocks), g, sms, st));
   // dx = dH W_gu (contract over the 2I interleaved rows)
-  g.scales = at<uint8_t>(wtp, LT.gu_scales); g.K = 2 * I; g.N = H; g.out0 = rows; g.hsaved = nullptr;
+  g.scales = at<uint8_t>(wtp, LT.gu_scales); g.K = 2 * I; g.N = H; g.out0 = rows; g.dgu = nullptr; g.act = nullptr;
   g.dw_part = nullptr;
   MOE_LAUNCH("gemm_dx_scatter", moe::launch_grouped_gemm(moe::kEpiDx, true, dh, at<uint8_t>(wtp, LT.gu_blocks), g, sms, st));
   MOE_LAUNCH("combine_dx", moe::launch_combine(rows, T, k, H, dx, st));
-  MOE_LAUNCH("router_backward", moe::launch_router_backward(idx, wr, inv, cbias, dwp, I / 32, T, E, k, d_topk_w, d_logits, st));
+  MOE_LAUNCH("reduce_dw", moe::launch_reduce_dw(cbias, dwp, I / 32, A, perm, dw, d_topk_w, st));
+  MOE_LAUNCH("router_backward", moe::launch_router_backward(idx, wr, d_topk_w, T, E, k, d_logits, st));
   return MXFP4_MOE_OK;
 }
 

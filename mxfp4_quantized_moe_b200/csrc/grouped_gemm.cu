@@ -45,9 +45,10 @@ namespace moe {
 
 namespace {
 
-constexpr int kTStages = 5;       // token ring depth
-constexpr int kWStages = 8;       // packed-weight ring depth (even: a stage keeps its parity)
-constexpr int kAStages = 4;       // TMEM A ring depth (even, same reason)
+// MMA-facing ring: stage s holds the token tile (shared memory) and the bf16 A operand
+// (TMEM) of one k-step; the MMA waits once and commits once per k-step.
+constexpr int kStages = 4;        // even: a stage always belongs to the same converter parity
+constexpr int kWStages = 8;       // packed-weight ring depth (even, same reason)
 constexpr int kThreads = 512;
 constexpr int kConvWarps = 8;
 constexpr int kTokBytes = kBN * kBK * 2;      // 24 KB
@@ -55,22 +56,29 @@ constexpr int kWBytes = kBM * (kBK / 2);      // 4 KB of packed nibbles
 constexpr int kAccCols = kBN;                 // fp32 accumulator columns per buffer
 constexpr int kACol0 = 2 * kAccCols;          // first TMEM column of the A ring
 constexpr int kTmemCols = 512;
-// registers per thread by warpgroup: control (producers, MMA), converters, epilogue
-constexpr int kRegsCtl = 56, kRegsConv = 128, kRegsEpi = 200;
-static_assert(128 * kRegsCtl + 256 * kRegsConv + 128 * kRegsEpi <= 65536, "register split");
-static_assert(kACol0 + kAStages * (kBK / 2) <= kTmemCols, "TMEM budget");
+// Registers per thread by warpgroup after setmaxnreg: control (producers, MMA, warpgroup 0),
+// converters (warpgroups 1-2), epilogue (warpgroup 3).  setmaxnreg.inc draws only on what the
+// other warpgroups released from the block's launch allocation (kThreads x kLaunchRegs), so
+// every warpgroup sets its count explicitly and the four shares must fit that allocation;
+// launch_one also refuses to launch if ptxas allocated fewer than kLaunchRegs per thread.
+constexpr int kLaunchRegs = 65536 / kThreads;  // 128: what __launch_bounds__(512, 1) allows
+constexpr int kRegsCtl = 56, kRegsConv = 112, kRegsEpi = 232;
+static_assert(kRegsCtl <= kLaunchRegs && kRegsConv <= kLaunchRegs && kRegsEpi >= kLaunchRegs,
+              "control and converter warpgroups only release registers; the epilogue takes");
+static_assert(128 * kRegsCtl + 2 * 128 * kRegsConv + 128 * kRegsEpi <= kThreads * kLaunchRegs,
+              "register split exceeds the block's launch allocation: setmaxnreg.inc would wait forever");
+static_assert(kRegsCtl % 8 == 0 && kRegsConv % 8 == 0 && kRegsEpi % 8 == 0, "setmaxnreg granularity");
+static_assert(kACol0 + kStages * (kBK / 2) <= kTmemCols, "TMEM budget");
 static_assert(kBN % 32 == 0 && kBN <= 256, "token tile");
-static_assert(kWStages % 2 == 0 && kAStages % 2 == 0, "ring depths must be even");
+static_assert(kWStages % 2 == 0 && kStages % 2 == 0, "ring depths must be even");
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 struct __align__(8) Barriers {
-  uint64_t t_full[kTStages];
-  uint64_t t_empty[kTStages];
+  uint64_t full[kStages];   // token bytes landed + 4 converter warps stored the A operand
+  uint64_t empty[kStages];  // MMA commit: token stage and A stage free again
   uint64_t w_full[kWStages];
   uint64_t w_empty[kWStages];
-  uint64_t a_full[kAStages];
-  uint64_t a_empty[kAStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t sc_full[2];
@@ -82,7 +90,7 @@ static_assert(sizeof(Barriers) <= 512, "barrier block");
 struct SmemLayout {
   // offsets from the 1024-aligned dynamic smem base
   static constexpr int tok = 0;                                  // 1024-aligned (128B swizzle)
-  static constexpr int w = tok + kTStages * kTokBytes;           // 256-aligned (32B swizzle)
+  static constexpr int w = tok + kStages * kTokBytes;            // 256-aligned (32B swizzle)
   static constexpr int bars = w + kWStages * kWBytes;
   static constexpr int misc = bars + 512;                        // tmem slot, abort flag
   static constexpr int cw = misc + 64;                           // 8 warps x 2 x 32 scale words
@@ -169,17 +177,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     *s_abort = 0;
     mbar_init(smem_u32(&bar->drain), 1);
-    for (int s = 0; s < kTStages; ++s) {
-      mbar_init(smem_u32(&bar->t_full[s]), 1);
-      mbar_init(smem_u32(&bar->t_empty[s]), 1);  // MMA commit
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&bar->full[s]), 1 + 4);  // token producer + 4 converter warps
+      mbar_init(smem_u32(&bar->empty[s]), 1);     // MMA commit
     }
     for (int s = 0; s < kWStages; ++s) {
       mbar_init(smem_u32(&bar->w_full[s]), 1);
       mbar_init(smem_u32(&bar->w_empty[s]), 4);  // the 4 converter warps of this parity
-    }
-    for (int s = 0; s < kAStages; ++s) {
-      mbar_init(smem_u32(&bar->a_full[s]), 4);
-      mbar_init(smem_u32(&bar->a_empty[s]), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bar->acc_full[s]), 1);
@@ -218,32 +222,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         prefetch_tmap(&tmap_tok);
         bool ok = true;
+        int s = 0;
+        uint32_t ph = 0;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
           Tile tl;
           decode_tile(t, s_tstart, s_off, E, nfb, tl);
           for (int ks = 0; ks < nk; ++ks) {
-            const int s = issued % kTStages;
-            if (!mbar_wait(smem_u32(&bar->t_empty[s]), ((issued / kTStages) & 1) ^ 1, err, 0x201,
-                           s_abort)) { ok = false; break; }
-            const uint32_t fb = smem_u32(&bar->t_full[s]);
+            if (!mbar_wait(smem_u32(&bar->empty[s]), ph ^ 1, err, 0x201, s_abort)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&bar->full[s]);
             mbar_arrive_expect_tx(fb, kTokBytes);
             tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
                         tl.row0, fb);
             ++issued;
+            if (++s == kStages) { s = 0; ph ^= 1; }
           }
         }
       }
       __syncwarp();
       __syncthreads();
-      // exit drain: every token copy issued has landed
-      if (lane == 0) drain_ring(bar->t_full, kTStages, issued, err, 0x2F0);
+      // exit drain: every token copy issued has landed.  `full` also counts converter
+      // arrivals, so wait on the copies' own completion: the stage's phase can only
+      // complete once its bytes are in (or the CTA aborted, which the drain bound covers).
+      if (lane == 0) drain_ring(bar->full, kStages, issued, err, 0x2F0);
     } else if (warp == 2) {
       // ============================ weight + scale producer =========================
       int issued = 0, sc_issued = 0;
       if (lane == 0) {
         prefetch_tmap(&tmap_w);
         bool ok = true;
-        int lt = 0;
+        int lt = 0, ws = 0;
+        uint32_t wph = 0;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
           Tile tl;
           decode_tile(t, s_tstart, s_off, E, nfb, tl);
@@ -263,14 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load(smem_u32(s_sc + sb * sc_bytes), src, bytes, smem_u32(&bar->sc_full[sb]));
           ++sc_issued;
           for (int ks = 0; ks < nk; ++ks) {
-            const int s = issued % kWStages;
-            if (!mbar_wait(smem_u32(&bar->w_empty[s]), ((issued / kWStages) & 1) ^ 1, err, 0x202,
-                           s_abort)) { ok = false; break; }
-            const uint32_t fb = smem_u32(&bar->w_full[s]);
+            if (!mbar_wait(smem_u32(&bar->w_empty[ws]), wph ^ 1, err, 0x202, s_abort)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&bar->w_full[ws]);
             mbar_arrive_expect_tx(fb, kWBytes);
-            tma_load_2d(smem_u32(smem + SmemLayout::w + s * kWBytes), &tmap_w, ks * (kBK / 2),
+            tma_load_2d(smem_u32(smem + SmemLayout::w + ws * kWBytes), &tmap_w, ks * (kBK / 2),
                         tl.e * N + tl.feat0, fb);
             ++issued;
+            if (++ws == kWStages) { ws = 0; wph ^= 1; }
           }
         }
       }
@@ -283,7 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ============================ MMA issuer ======================================
       if (lane == 0) {
-        int g = 0;  // k-steps issued so far (all tiles)
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t tok_addr = smem_u32(smem + SmemLayout::tok);
+        uint32_t a_tmem = tmem + kACol0;
         int lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
@@ -294,23 +304,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t idesc = idesc_bf16_m128((tl.n_valid + 15) & ~15);
           const uint32_t d_tmem = tmem + acc * kAccCols;
-          for (int ks = 0; ks < nk; ++ks, ++g) {
-            const int s = g % kTStages, sa = g % kAStages;
-            if (!mbar_wait(smem_u32(&bar->t_full[s]), (g / kTStages) & 1, err, 0x301, s_abort) ||
-                !mbar_wait(smem_u32(&bar->a_full[sa]), (g / kAStages) & 1, err, 0x302, s_abort)) {
+          for (int ks = 0; ks < nk; ++ks) {
+            if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t bdesc =
-                smem_desc_kmajor_sw128(smem_u32(smem + SmemLayout::tok + s * kTokBytes));
-            const uint32_t a_tmem = tmem + kACol0 + sa * (kBK / 2);
+            const uint64_t bdesc = smem_desc_kmajor_sw128(tok_addr);
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk)
               mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
                           (ks | kk) != 0);
-            mma_commit(smem_u32(&bar->t_empty[s]));
-            mma_commit(smem_u32(&bar->a_empty[sa]));
+            mma_commit(smem_u32(&bar->empty[s]));
+            if (++s == kStages) {
+              s = 0;
+              ph ^= 1;
+              tok_addr = smem_u32(smem + SmemLayout::tok);
+              a_tmem = tmem + kACol0;
+            } else {
+              tok_addr += kTokBytes;
+              a_tmem += kBK / 2;
+            }
           }
           if (ok) mma_commit(smem_u32(&bar->acc_full[acc]));
         }
@@ -325,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (wg < 3) {
     // ================================ converters ====================================
+    if (kRegsConv < kLaunchRegs) setmaxnreg_dec<kRegsConv>();
     // Converter warp c (0..7) serves TMEM lane quarter q = warp % 4 and the k-steps whose
     // running index g has parity c / 4; its partner warp takes the other parity.
     const int q = warp & 3;
@@ -427,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        const int sa = g % kAStages;
-        if (!mbar_wait(smem_u32(&bar->a_empty[sa]), ((g / kAStages) & 1) ^ 1, err, 0x402,
+        const int sa = g % kStages;
+        if (!mbar_wait(smem_u32(&bar->empty[sa]), ((g / kStages) & 1) ^ 1, err, 0x402,
                        s_abort)) {
           ok = false;
           break;
@@ -440,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();  // also orders this k-step's reads of cw before the next writes
-        if (lane == 0) mbar_arrive(smem_u32(&bar->a_full[sa]));
+        if (lane == 0) mbar_arrive(smem_u32(&bar->full[sa]));
       }
       if (!ok) break;
       __syncwarp();
@@ -457,10 +472,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       Tile tl;
       decode_tile(t, s_tstart, s_off, E, nfb, tl);
       const int acc = lt & 1;
-      if (!mbar_wait(smem_u32(&bar->acc_full[acc]), (lt >> 1) & 1, err, 0x500, s_abort)) break;
-      tc_fence_after();
       const int f = tl.feat0 + 32 * q + lane;  // output feature of this thread
       const bool active = tl.feat0 + 32 * q < N;
+      // dact: the saved GLU factors and act of the tile's first 32 rows are requested before
+      // the accumulator is ready; each chunk then requests the next chunk's while it computes
+      uint32_t dnext[32];
+      uint16_t anext[32];
+      if (EPI == kEpiDact && active) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const size_t o = (size_t)min(tl.row0 + j, p.A - 1) * N + f;
+          dnext[j] = __ldg(p.dgu + o);
+          anext[j] = __ldg(p.act + o);
+        }
+      }
+      if (!mbar_wait(smem_u32(&bar->acc_full[acc]), (lt >> 1) & 1, err, 0x500, s_abort)) break;
+      tc_fence_after();
       float bias_f = 0.f;
       if ((EPI == kEpiGateUp || EPI == kEpiDown) && active)
         bias_f = bf16_to_f(p.bias[(size_t)tl.e * N + f]);
@@ -475,10 +502,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (EPI == kEpiGateUp) {
           // Columns j (even lane) and j+1 (odd lane) of each pair: the lanes of an
           // interleaved (gate, up) feature pair swap one value so that each holds (g, u) of
-          // its own column; it stores h as one bf16x2 word and act as one bf16.
+          // its own column.  Stored per (row, j): act = (u'+1) g' sigmoid(a g') and, for the
+          // backward, the GLU derivative factors d act/d g and d act/d u as one bf16x2 word
+          // (clamp masks decided on h rounded to bf16, as the eager bf16 model holds it).
           const int I = N >> 1;
           const int jf = f >> 1;
-          uint32_t hw[16];
+          uint32_t dw16[16];
           float av[16];
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
@@ -487,18 +516,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float recv = __shfl_xor_sync(kFull, odd ? v0 : v1, 1);
             const float g = odd ? recv : v0;
             const float u = odd ? v1 : recv;
-            hw[jj] = pack_bf16x2(g, u);
             const float gc = fminf(g, p.limit);
             const float uc = fminf(fmaxf(u, -p.limit), p.limit);
-            av[jj] = (uc + 1.f) * gc * fast_sigmoid(p.alpha * gc);
+            const float sg = fast_sigmoid(p.alpha * gc);
+            const float t1 = gc * sg;
+            const float up1 = uc + 1.f;
+            av[jj] = up1 * t1;
+            const float gb = bf16_to_f(f_to_bf16(g)), ub = bf16_to_f(f_to_bf16(u));
+            const float dgc = (gb <= p.limit) ? up1 * (sg + p.alpha * t1 * (1.f - sg)) : 0.f;
+            const float duc = (ub >= -p.limit && ub <= p.limit) ? t1 : 0.f;
+            dw16[jj] = pack_bf16x2(dgc, duc);
           }
-          uint32_t* hrow = reinterpret_cast<uint32_t*>(p.out0);
+          uint32_t* dgu_out = reinterpret_cast<uint32_t*>(p.out0);
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int col = 2 * jj + (odd ? 1 : 0);
             if (col < ncol) {
-              hrow[((size_t)(rbase + col) * N + (f & ~1)) >> 1] = hw[jj];
-              p.out1[(size_t)(rbase + col) * I + jf] = f_to_bf16(av[jj]);
+              const size_t o = (size_t)(rbase + col) * I + jf;
+              dgu_out[o] = dw16[jj];
+              p.out1[o] = f_to_bf16(av[jj]);
             }
           }
         } else {
@@ -531,37 +567,35 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (col < ncol) orow[((size_t)slot * N + (f & ~1)) >> 1] = ow[jj];
             }
           } else {  // kEpiDact
+            // dZ = dY W_d for this row; dact = w dZ; dH = (dact * dact/dg, dact * dact/du)
+            // from the factors the forward saved; partial <dZ, act> for the routing gradient.
             const int I = N;
-            const uint32_t* hw = reinterpret_cast<const uint32_t*>(p.hsaved);
             uint32_t* dh = reinterpret_cast<uint32_t*>(p.out0);
-            // issue all 32 loads of the saved (g, u) pairs first (h is read-only here);
-            // columns past the tile's rows read a valid row and are discarded
-            uint32_t hv[32];
+            uint32_t dcur[32];
+            uint16_t acur[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const int row = min(rbase + j, p.A - 1);
-              hv[j] = __ldg(hw + (size_t)row * I + f);
+              dcur[j] = dnext[j];
+              acur[j] = anext[j];
+            }
+            if (c0 + 32 < tl.n_valid) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const size_t o = (size_t)min(rbase + 32 + j, p.A - 1) * I + f;
+                dnext[j] = __ldg(p.dgu + o);
+                anext[j] = __ldg(p.act + o);
+              }
             }
             float part[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float wr = __shfl_sync(kFull, my_w, j);
-              const float g = bf16_lo(hv[j]), u = bf16_hi(hv[j]);
               const float dz = __uint_as_float(r[j]);
-              const float gc = fminf(g, p.limit);
-              const float uc = fminf(fmaxf(u, -p.limit), p.limit);
-              const float sg = fast_sigmoid(p.alpha * gc);
-              part[j] = (j < ncol) ? dz * ((uc + 1.f) * gc * sg) : 0.f;
+              part[j] = (j < ncol) ? dz * bf16_to_f(acur[j]) : 0.f;
               const float dact = wr * dz;
-              const float dg = (g <= p.limit)
-                                   ? dact * (uc + 1.f) * (sg + p.alpha * gc * sg * (1.f - sg))
-                                   : 0.f;
-              const float du = (u >= -p.limit && u <= p.limit) ? dact * gc * sg : 0.f;
-              hv[j] = pack_bf16x2(dg, du);
+              const uint32_t dh2 = pack_bf16x2(dact * bf16_lo(dcur[j]), dact * bf16_hi(dcur[j]));
+              if (j < ncol) dh[(size_t)(rbase + j) * I + f] = dh2;
             }
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < ncol) dh[(size_t)(rbase + j) * I + f] = hv[j];
             const float sum = warp_transpose_reduce(part, lane);
             if (lane < ncol) p.dw_part[(size_t)((tl.feat0 >> 5) + q) * p.A + rbase + lane] = sum;
           }
@@ -605,6 +639,11 @@ template <int EPI, bool COLT>
 cudaError_t launch_one(const CUtensorMap& tt, const CUtensorMap& tw, const GemmArgs& a, int grid,
                        size_t smem, cudaStream_t st) {
   auto kern = grouped_gemm_kernel<EPI, COLT>;
+  // the setmaxnreg split assumes kLaunchRegs registers per thread at launch
+  cudaFuncAttributes fa;
+  cudaError_t fe = cudaFuncGetAttributes(&fa, kern);
+  if (fe != cudaSuccess) return fe;
+  if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

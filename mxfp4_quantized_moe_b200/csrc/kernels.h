@@ -21,9 +21,10 @@ struct GemmArgs {
   const int32_t* off;      // [E+1] start row of each expert in the expert-sorted order
   int E, K, N, A;          // experts, contraction length, output features, assignments
   const uint16_t* bias;    // bf16 [E][N]: gate_up bias (kEpiGateUp) or down bias (kEpiDown)
-  uint16_t* out0;          // h [A][2I] | Yslot [A][H] | dH [A][2I] | dXslot [A][H]
+  uint16_t* out0;          // dGU [A][I] (bf16x2) | Yslot [A][H] | dH [A][2I] | dXslot [A][H]
   uint16_t* out1;          // act [A][I] (kEpiGateUp)
-  const uint16_t* hsaved;  // h [A][2I] (kEpiDact)
+  const uint32_t* dgu;     // saved GLU derivative factors [A][I] bf16x2 (kEpiDact)
+  const uint16_t* act;     // saved act [A][I] bf16 (kEpiDact)
   const int32_t* perm;     // [A] sorted row -> slot t*k+j
   const float* topk_w;     // [A] routing weight per slot
   float* dw_part;          // [N/32][A] partial <dZ, act> sums (kEpiDact)
@@ -48,10 +49,12 @@ cudaError_t launch_gather_rows(const uint16_t* src, int H, int k, const int32_t*
                                float* dot_out, cudaStream_t st);
 cudaError_t launch_combine(const uint16_t* slots, int T, int k, int H, uint16_t* out,
                            cudaStream_t st);
-cudaError_t launch_router_backward(const int32_t* idx, const float* w, const int32_t* inv,
-                                   const float* cbias, const float* dw_part, int nparts, int T,
-                                   int E, int k, float* d_topk_w, float* d_logits,
-                                   cudaStream_t st);
+// dw[r] = cbias[r] + sum_p dw_part[p][r]; d_topk_w[perm[r]] = dw[r]  (one thread per row)
+cudaError_t launch_reduce_dw(const float* cbias, const float* dw_part, int nparts, int A,
+                             const int32_t* perm, float* dw, float* d_topk_w, cudaStream_t st);
+// d_logits from d_topk_w through the softmax over the k selected logits (one thread per token)
+cudaError_t launch_router_backward(const int32_t* idx, const float* w, const float* d_topk_w,
+                                   int T, int E, int k, float* d_logits, cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
                            uint16_t* out, cudaStream_t st);
 cudaError_t launch_transpose_packed(const uint8_t* src, int E, int R, int C, uint8_t* dst,

@@ -195,35 +195,35 @@ __global__ void combine_kernel(const uint16_t* __restrict__ slots, int T, int k,
   reinterpret_cast<uint4*>(out + (size_t)t * H)[c] = o;
 }
 
-// d_topk_w[t,j] = cbias[r] + sum_p dw_part[p][r] (r = inv[t*k+j]); d_logits through the
-// softmax over the k selected logits: d_l[idx_j] = w_j (d_w_j - sum_i w_i d_w_i), 0 elsewhere.
+// Routing-weight gradient per expert-sorted row: dw[r] = <dY_t, b_d[e]> + sum of the GEMM's
+// per-32-feature partial <dZ_r, act_r>; written to its slot.  Reads of the [P][A] partials
+// are coalesced across threads (consecutive rows).
+__global__ void reduce_dw_kernel(const float* __restrict__ cbias, const float* __restrict__ dw_part,
+                                 int nparts, int A, const int32_t* __restrict__ perm,
+                                 float* __restrict__ dw, float* __restrict__ d_topk_w) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= A) return;
+  float v = cbias[r];
+  for (int q = 0; q < nparts; ++q) v += __ldg(dw_part + (size_t)q * A + r);
+  dw[r] = v;
+  d_topk_w[perm[r]] = v;
+}
+
+// d_logits through the softmax over the k selected logits:
+// d_l[idx_j] = w_j (d_w_j - sum_i w_i d_w_i), 0 for the experts not selected.
 __global__ void router_backward_kernel(const int32_t* __restrict__ idx,
                                        const float* __restrict__ w,
-                                       const int32_t* __restrict__ inv,
-                                       const float* __restrict__ cbias,
-                                       const float* __restrict__ dw_part, int nparts, int A,
-                                       int T, int E, int k, float* __restrict__ d_topk_w,
+                                       const float* __restrict__ d_topk_w, int T, int E, int k,
                                        float* __restrict__ d_logits) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
-  float dw[16];
   float s = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const int slot = t * k + j;
-    const int r = inv[slot];
-    float v = cbias[r];
-    for (int p = 0; p < nparts; ++p) v += dw_part[(size_t)p * A + r];
-    d_topk_w[slot] = v;
-    if (j < 16) dw[j] = v;
-    s += w[slot] * v;
-  }
-  if (!d_logits) return;
+  for (int j = 0; j < k; ++j) s += w[t * k + j] * d_topk_w[t * k + j];
   float* dl = d_logits + (size_t)t * E;
   for (int e = 0; e < E; ++e) dl[e] = 0.f;
   for (int j = 0; j < k; ++j) {
     const int slot = t * k + j;
-    const float v = (j < 16) ? dw[j] : d_topk_w[slot];
-    dl[idx[slot]] = w[slot] * (v - s);
+    dl[idx[slot]] = w[slot] * (d_topk_w[slot] - s);
   }
 }
 
@@ -326,12 +326,16 @@ cudaError_t launch_combine(const uint16_t* slots, int T, int k, int H, uint16_t*
   return cudaGetLastError();
 }
 
-cudaError_t launch_router_backward(const int32_t* idx, const float* w, const int32_t* inv,
-                                   const float* cbias, const float* dw_part, int nparts, int T,
-                                   int E, int k, float* d_topk_w, float* d_logits,
-                                   cudaStream_t st) {
-  router_backward_kernel<<<(T + 127) / 128, 128, 0, st>>>(idx, w, inv, cbias, dw_part, nparts,
-                                                          T * k, T, E, k, d_topk_w, d_logits);
+cudaError_t launch_reduce_dw(const float* cbias, const float* dw_part, int nparts, int A,
+                             const int32_t* perm, float* dw, float* d_topk_w, cudaStream_t st) {
+  reduce_dw_kernel<<<(A + 255) / 256, 256, 0, st>>>(cbias, dw_part, nparts, A, perm, dw, d_topk_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_backward(const int32_t* idx, const float* w, const float* d_topk_w,
+                                   int T, int E, int k, float* d_logits, cudaStream_t st) {
+  if (!d_logits) return cudaSuccess;
+  router_backward_kernel<<<(T + 127) / 128, 128, 0, st>>>(idx, w, d_topk_w, T, E, k, d_logits);
   return cudaGetLastError();
 }
 
