@@ -35,7 +35,7 @@ DEFAULT_WORKLOAD = "gpt-oss-20b-moe-T8192"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -181,7 +181,7 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from mxfp4_quantized_moe_b200 import inputs, moe
+    from mxfp4_quantized_moe_b200 import inputs, moe, replicas
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -192,10 +192,10 @@ def main():
     wl = inputs.WORKLOADS[args.workload]
     if wl.layers != 1:
         raise SystemExit("bench times single-layer workloads")
-    # each rank draws its own batch (seed + rank); the weights are the same on every rank
+    # each rank draws its own token batch; the weights are the same on every rank
     inp = inputs.make_workload(wl, args.seed)
     if rank:
-        xr = inputs.make_workload(wl, args.seed + 1000 * rank)
+        xr = inputs.make_workload(wl, replicas.batch_seed(args.seed, rank))
         inp = dict(inp, x=xr["x"], logits=xr["logits"], dy=xr["dy"])
     shape = moe.MoeShape(wl.T, wl.H, wl.I, wl.E, wl.k)
     w = moe.weights_to(inp, dev)
@@ -243,10 +243,7 @@ def main():
     rc, where = moe.device_check(ws)
     if rc != 0:
         raise SystemExit(f"device error {rc} at {where:#x}")
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = replicas.max_over_ranks(ms, dev)
 
     # ---- end to end through the public API with host buffers ----------------------------
     hx = inp["x"].pin_memory()
@@ -276,10 +273,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    t2 = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t2.item())
+    e2e_ms = replicas.max_over_ranks(e0.elapsed_time(e1), dev)
     h2d = sum(int(v.numel() * v.element_size()) for v in (hx, hlg, hdy))
     d2h = sum(int(v.numel() * v.element_size()) for v in (hy, hdx, hdtw, hdl))
 
@@ -292,7 +286,7 @@ def main():
     T, H, I, E, k = wl.T, wl.H, wl.I, wl.E, wl.k
     A = T * k
     flop_step = 12.0 * A * H * I
-    value = T * world * args.steps / (ms_max / 1e3)
+    value = replicas.aggregate_tokens_per_s(T, args.steps, ms_max, world)
     pk = peaks()
     # dominant kernel: largest summed device time inside the timed region
     gemm_flops = {"gemm_gate_up_glu": 2.0 * A * H * 2 * I, "gemm_down_scatter": 2.0 * A * I * H,
@@ -336,7 +330,8 @@ def main():
                    / pk["bf16_tflops_sustained"]},
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": T * world * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": replicas.aggregate_tokens_per_s(T, args.e2e_steps, e2e_ms, world),
+                "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_total,
         "kernels": kernel_table,

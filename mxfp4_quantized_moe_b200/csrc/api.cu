@@ -1,5 +1,6 @@
 // C ABI of the MXFP4 MoE expert block: argument checks, workspace carving and the launch
 // sequence of the forward and input-gradient backward.  See include/mxfp4_moe.h.
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <vector>
@@ -90,6 +91,26 @@ int check_device(int* sms) {
   if (sms && cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MXFP4_MOE_ERR_CUDA;
   return MXFP4_MOE_OK;
+}
+
+// Largest fp32 x such that bf16(x) <= limit under round-to-nearest-even: the clamp-mask
+// decision "bf16(h) <= limit" becomes one fp32 compare.  For limit = 7 this is 7.015625
+// (the tie between 7 and the next bf16, 7.03125, rounds to 7, whose mantissa is even).
+float bf16_mask_limit(float limit) {
+  uint32_t b;
+  std::memcpy(&b, &limit, 4);
+  // largest bf16 value <= limit (truncate the fp32 pattern toward zero for positive limits)
+  uint32_t lo = b & 0xFFFF0000u;
+  float flo;
+  std::memcpy(&flo, &lo, 4);
+  const uint32_t hi = lo + 0x10000u;  // next bf16 up
+  float fhi;
+  std::memcpy(&fhi, &hi, 4);
+  const double mid = 0.5 * ((double)flo + (double)fhi);  // exact in fp32 (one extra bit)
+  float m = (float)mid;
+  const bool lo_even = ((lo >> 16) & 1u) == 0;
+  if (!lo_even) m = std::nextafter(m, 0.0f);  // a tie would round up to the odd neighbour... of hi
+  return m;
 }
 
 #define MOE_TRY(expr)                                  \
@@ -226,7 +247,7 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
 
   moe::GemmArgs g{};
   g.off = off; g.E = E; g.A = A; g.perm = perm; g.topk_w = wr; g.err = err;
-  g.alpha = d->glu_alpha; g.limit = d->glu_limit;
+  g.alpha = d->glu_alpha; g.limit = d->glu_limit; g.mask_limit = bf16_mask_limit(d->glu_limit);
   // gate_up: h = Xp W_gu^T + b_gu; act = GLU(h) and the GLU derivative factors are saved
   g.scales = w->gu_scales; g.K = H; g.N = 2 * I; g.bias = w->gu_bias; g.out0 = dgu; g.out1 = act;
   MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, rows, w->gu_blocks, g, sms, st));

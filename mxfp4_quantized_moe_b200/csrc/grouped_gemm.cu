@@ -108,6 +108,19 @@ struct Tile {
   int e, fb, row0, n_valid, feat0;
 };
 
+// An expert's m rows are split into equal token tiles of at most kBN rows (a multiple of 16),
+// so that no tile is a small remainder: the MMA costs nearly the same at N = 64 as at N = 192.
+MOE_DEV int token_tile_rows(int m) {
+  const int n = (m + kBN - 1) / kBN;
+  const int rows = (m + n - 1) / n;
+  return (rows + 15) & ~15;
+}
+MOE_DEV int token_tiles(int m) {
+  if (m <= 0) return 0;
+  const int rows = token_tile_rows(m);
+  return (m + rows - 1) / rows;
+}
+
 __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const int* s_off, int E,
                                             int nfb, Tile& o) {
   int lo = 0, hi = E;  // largest lo with s_tstart[lo] <= t (s_tstart[E] = total > t)
@@ -117,10 +130,12 @@ __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const in
   }
   const int local = t - s_tstart[lo];
   const int tt = local / nfb;
+  const int m = s_off[lo + 1] - s_off[lo];
+  const int rows = token_tile_rows(m);
   o.e = lo;
   o.fb = local - tt * nfb;
-  o.row0 = s_off[lo] + tt * kBN;
-  o.n_valid = min(kBN, s_off[lo + 1] - o.row0);
+  o.row0 = s_off[lo] + tt * rows;
+  o.n_valid = min(rows, m - tt * rows);
   o.feat0 = o.fb * kBM;
 }
 
@@ -202,8 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       s_tstart[e] = acc;
-      const int m = s_off[e + 1] - s_off[e];
-      acc += ((m + kBN - 1) / kBN) * nfb;
+      acc += token_tiles(s_off[e + 1] - s_off[e]) * nfb;
     }
     s_tstart[E] = acc;
   }
@@ -292,8 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         int s = 0;
         uint32_t ph = 0;
-        uint32_t tok_addr = smem_u32(smem + SmemLayout::tok);
-        uint32_t a_tmem = tmem + kACol0;
+        const uint32_t tok_base = smem_u32(smem + SmemLayout::tok);
         int lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
@@ -304,26 +317,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t idesc = idesc_bf16_m128((tl.n_valid + 15) & ~15);
           const uint32_t d_tmem = tmem + acc * kAccCols;
-          for (int ks = 0; ks < nk; ++ks) {
-            if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort)) {
+          // Two k-steps per round: both stages are waited for first, then their eight MMAs
+          // go out back to back (the issuing thread blocks while the tensor pipe is busy, so
+          // the bookkeeping between rounds is the only gap the pipe can see).
+          for (int ks = 0; ks < nk; ks += 2) {
+            const bool two = ks + 1 < nk;
+            const int s1 = (s + 1 == kStages) ? 0 : s + 1;
+            const uint32_t ph1 = (s + 1 == kStages) ? (ph ^ 1) : ph;
+            if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort) ||
+                (two && !mbar_wait(smem_u32(&bar->full[s1]), ph1, err, 0x301, s_abort))) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t bdesc = smem_desc_kmajor_sw128(tok_addr);
+            {
+              const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + s * kTokBytes);
+              const uint32_t a_tmem = tmem + kACol0 + s * (kBK / 2);
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-              mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
-                          (ks | kk) != 0);
-            mma_commit(smem_u32(&bar->empty[s]));
-            if (++s == kStages) {
-              s = 0;
-              ph ^= 1;
-              tok_addr = smem_u32(smem + SmemLayout::tok);
-              a_tmem = tmem + kACol0;
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
+                            (ks | kk) != 0);
+              mma_commit(smem_u32(&bar->empty[s]));
+            }
+            if (two) {
+              const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + s1 * kTokBytes);
+              const uint32_t a_tmem = tmem + kACol0 + s1 * (kBK / 2);
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc, 1u);
+              mma_commit(smem_u32(&bar->empty[s1]));
+              s = (s1 + 1 == kStages) ? 0 : s1 + 1;
+              ph = (s1 + 1 == kStages) ? (ph1 ^ 1) : ph1;
             } else {
-              tok_addr += kTokBytes;
-              a_tmem += kBK / 2;
+              s = s1;
+              ph = ph1;
             }
           }
           if (ok) mma_commit(smem_u32(&bar->acc_full[acc]));
@@ -522,9 +549,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float t1 = gc * sg;
             const float up1 = uc + 1.f;
             av[jj] = up1 * t1;
-            const float gb = bf16_to_f(f_to_bf16(g)), ub = bf16_to_f(f_to_bf16(u));
-            const float dgc = (gb <= p.limit) ? up1 * (sg + p.alpha * t1 * (1.f - sg)) : 0.f;
-            const float duc = (ub >= -p.limit && ub <= p.limit) ? t1 : 0.f;
+            // bf16(g) <= limit  <=>  g <= mask_limit (and likewise for |bf16(u)|)
+            const float dgc = (g <= p.mask_limit) ? up1 * (sg + p.alpha * t1 * (1.f - sg)) : 0.f;
+            const float duc = (fabsf(u) <= p.mask_limit) ? t1 : 0.f;
             dw16[jj] = pack_bf16x2(dgc, duc);
           }
           uint32_t* dgu_out = reinterpret_cast<uint32_t*>(p.out0);

@@ -29,6 +29,7 @@ struct GemmArgs {
   const float* topk_w;     // [A] routing weight per slot
   float* dw_part;          // [N/32][A] partial <dZ, act> sums (kEpiDact)
   float alpha, limit;
+  float mask_limit;        // largest fp32 x whose bf16 rounding is <= limit (clamp-mask test)
   int* err;
 };
 
