@@ -15,6 +15,7 @@ of each step's workload, on this host's cores.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -55,6 +56,30 @@ def peaks():
                 "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a grouped GEMM,
+# from an ncu capture of this bench's workload; summaries under profiles/.  An entry counts
+# only while the kernel's sources hash to `sources`: after any change it reads as null.
+NCU_TRAFFIC = {}
+KERNEL_SOURCES = ("mxfp4_quantized_moe_b200/csrc/grouped_gemm.cu",
+                  "mxfp4_quantized_moe_b200/csrc/common.cuh",
+                  "mxfp4_quantized_moe_b200/csrc/kernels.h")
+
+
+def kernel_sources_digest():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    e = NCU_TRAFFIC.get((kernel, workload))
+    if e is None or e["sources"] != kernel_sources_digest():
+        return None
+    return e["bytes"]
 
 
 def cpu_threads():
@@ -299,7 +324,8 @@ def main():
         achieved = gemm_flops[name] / (avg_ms / 1e3) / 1e12
         peak = pk["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": name,
+                "frac": achieved / peak, "traffic": recorded_traffic(name, wl.name),
+                "traffic_unit": "bytes per launch (ncu DRAM read+write)", "kernel": name,
                 "avg_launch_ms": avg_ms,
                 "peak_source": f"{pk['source']} bf16 sustained (kernel timed inside a long step)"}
     launches_total = sum(v[0] for v in kt.values())
