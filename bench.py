@@ -82,6 +82,26 @@ def recorded_traffic(kernel, workload):
     return e["bytes"]
 
 
+def gemm_work(wl):
+    """Algorithmic FLOP and DRAM bytes of one launch of each grouped GEMM: every operand read
+    once and every result written once (packed MXFP4 weights at 0.5 B per element plus one
+    scale byte per 32, bf16 activations, saved GLU factors at 4 B per (row, j))."""
+    T, H, I, E, k = wl.T, wl.H, wl.I, wl.E, wl.k
+    A = T * k
+    w_gu = E * 2 * I * H * (0.5 + 1 / 32)  # packed gate_up (or its transposed copy)
+    w_dn = E * H * I * (0.5 + 1 / 32)
+    return {
+        "gemm_gate_up_glu": (2.0 * A * H * 2 * I,
+                             w_gu + E * 2 * I * 2 + A * H * 2 + A * I * (4 + 2)),
+        "gemm_down_scatter": (2.0 * A * I * H,
+                              w_dn + E * H * 2 + A * I * 2 + A * 8 + A * H * 2),
+        "gemm_dact_glu_bwd": (2.0 * A * H * I,
+                              w_dn + A * H * 2 + A * I * (4 + 2) + A * 4 + A * 2 * I * 2
+                              + A * (I // 32) * 4),
+        "gemm_dx_scatter": (2.0 * A * 2 * I * H, w_gu + A * 2 * I * 2 + A * H * 2),
+    }
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -314,20 +334,30 @@ def main():
     value = replicas.aggregate_tokens_per_s(T, args.steps, ms_max, world)
     pk = peaks()
     # dominant kernel: largest summed device time inside the timed region
-    gemm_flops = {"gemm_gate_up_glu": 2.0 * A * H * 2 * I, "gemm_down_scatter": 2.0 * A * I * H,
-                  "gemm_dact_glu_bwd": 2.0 * A * H * I, "gemm_dx_scatter": 2.0 * A * 2 * I * H}
+    work = gemm_work(wl)
     top = max(kt.items(), key=lambda kv: kv[1][1])
     name, (launches, tot) = top
     roof = None
-    if name in gemm_flops:
+    if name in work:
         avg_ms = tot / launches
-        achieved = gemm_flops[name] / (avg_ms / 1e3) / 1e12
-        peak = pk["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(name, wl.name),
-                "traffic_unit": "bytes per launch (ncu DRAM read+write)", "kernel": name,
-                "avg_launch_ms": avg_ms,
-                "peak_source": f"{pk['source']} bf16 sustained (kernel timed inside a long step)"}
+        flops, nbytes = work[name]
+        ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+        roof = {"kernel": name, "avg_launch_ms": avg_ms, "algorithmic_flop": flops,
+                "algorithmic_bytes": nbytes, "intensity_flop_per_byte": flops / nbytes,
+                "ridge_flop_per_byte": ridge,
+                "traffic": recorded_traffic(name, wl.name),
+                "traffic_unit": "bytes per launch (ncu DRAM read+write)"}
+        if flops / nbytes >= ridge:
+            achieved = flops / (avg_ms / 1e3) / 1e12
+            peak = pk["bf16_tflops_sustained"]
+            roof.update(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
+                        frac=achieved / peak, peak_source=f"{pk['source']} bf16 sustained "
+                        "(kernel timed inside a long step)")
+        else:  # few rows per expert: bound by streaming the packed weights
+            achieved = nbytes / (avg_ms / 1e3) / 1e9
+            peak = pk["hbm_gbs"]
+            roof.update(bound="hbm", achieved=achieved, peak=peak, unit="GB/s",
+                        frac=achieved / peak, peak_source=f"{pk['source']} HBM copy bandwidth")
     launches_total = sum(v[0] for v in kt.values())
     kernel_table = {kname: {"launches": v[0], "ms_per_launch": v[1] / v[0],
                             "share": v[1] / sum(u[1] for u in kt.values())} for kname, v in kt.items()}

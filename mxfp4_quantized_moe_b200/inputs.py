@@ -45,6 +45,8 @@ WORKLOADS = {
     "gpt-oss-20b-moe-T8192": Workload("gpt-oss-20b-moe-T8192", 8192, 2880, 2880, 32, 4),
     # smaller batch of the same layer, for profiler captures that must stay a few GB
     "gpt-oss-20b-moe-T4096": Workload("gpt-oss-20b-moe-T4096", 4096, 2880, 2880, 32, 4),
+    # small-token case: ~32 rows per expert, bound by streaming the packed weights
+    "gpt-oss-20b-moe-T256": Workload("gpt-oss-20b-moe-T256", 256, 2880, 2880, 32, 4),
     "gpt-oss-120b-moe-T16384": Workload("gpt-oss-120b-moe-T16384", 16384, 2880, 2880, 128, 4),
     "gpt-oss-20b-moe-zipf-T16384": Workload("gpt-oss-20b-moe-zipf-T16384", 16384, 2880, 2880, 32, 4,
                                             zipf_s=1.2),

@@ -222,6 +222,17 @@ def _expert_weights(W, e):
     return wgu, wd
 
 
+def _weights_of(W, e):
+    """Dequantized weights of expert e.  When the caller puts a dict under
+    W["_dequant_cache"], each expert is dequantized once and reused (same values)."""
+    cache = W.get("_dequant_cache")
+    if cache is None:
+        return _expert_weights(W, e)
+    if e not in cache:
+        cache[e] = _expert_weights(W, e)
+    return cache[e]
+
+
 def moe_forward(x, logits, W, k: int, alpha: float = 1.702, limit: float = 7.0):
     """Forward of the expert block.
 
@@ -245,7 +256,7 @@ def moe_forward(x, logits, W, k: int, alpha: float = 1.702, limit: float = 7.0):
         tt, jj = np.nonzero(idx == e)  # slot order t*k + j
         if tt.size == 0:
             continue
-        wgu, wd = _expert_weights(W, e)
+        wgu, wd = _weights_of(W, e)
         h = x[tt] @ wgu.T + gu_bias[e]
         act = glu(h, alpha, limit)
         y = act @ wd.T + dn_bias[e]
@@ -272,7 +283,7 @@ def moe_backward(dY, fwd, W, alpha: float = 1.702, limit: float = 7.0):
         tt, jj = np.nonzero(idx == e)
         if tt.size == 0:
             continue
-        wgu, wd = _expert_weights(W, e)
+        wgu, wd = _weights_of(W, e)
         dy = w[tt, jj][:, None] * dY[tt]
         dact = dy @ wd  # [n, I]
         h = fwd["h"][tt, jj]
@@ -286,3 +297,37 @@ def moe_backward(dY, fwd, W, alpha: float = 1.702, limit: float = 7.0):
     d_logits = np.zeros((T, E), dtype=np.float64)
     np.put_along_axis(d_logits, idx, d_sel, axis=1)
     return dX, d_w, d_logits
+
+
+# --------------------------------------------------------------------------------------
+# Residual stack of blocks (the caller's side: router linear and residual add)
+# --------------------------------------------------------------------------------------
+def stack_forward(x, layers, k: int, alpha: float = 1.702, limit: float = 7.0):
+    """x_{l+1} = x_l + block_l(x_l, logits_l), logits_l = x_l W_r^l + b_r^l, all in fp64.
+
+    layers: list of dicts {"W": block weights as for moe_forward, "w_r": [H,E], "b_r": [E]}.
+    Returns (x_L, records) with records[l] = {"x": x_l, "logits": logits_l, "fwd": ...}.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    recs = []
+    for L in layers:
+        logits = x @ np.asarray(L["w_r"], np.float64) + np.asarray(L["b_r"], np.float64)
+        f = moe_forward(x, logits, L["W"], k, alpha, limit)
+        recs.append({"x": x, "logits": logits, "fwd": f})
+        x = x + f["out"]
+    return x, recs
+
+
+def stack_backward(dY, recs, layers, alpha: float = 1.702, limit: float = 7.0):
+    """dL/dx_0 of the stack: walking the blocks backwards, the gradient of block l's input
+    is the residual path plus the block's input gradient plus the router path,
+        g_l = g_{l+1} + dX_l + d_logits_l (W_r^l)^T,
+    where (dX_l, d_logits_l) are the block's input gradients for upstream g_{l+1}.
+    Returns (g_0, per-layer (g_{l+1}, dX_l, d_w_l, d_logits_l), in layer order)."""
+    g = np.asarray(dY, dtype=np.float64)
+    per = [None] * len(layers)
+    for l in range(len(layers) - 1, -1, -1):
+        dX, d_w, d_logits = moe_backward(g, recs[l]["fwd"], layers[l]["W"], alpha, limit)
+        per[l] = (g, dX, d_w, d_logits)
+        g = g + dX + d_logits @ np.asarray(layers[l]["w_r"], np.float64).T
+    return g, per

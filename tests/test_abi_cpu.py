@@ -113,3 +113,15 @@ def test_python_wrappers_have_no_cpu_path():
     from mxfp4_quantized_moe_b200 import moe
     with pytest.raises(ValueError):
         moe.dequantize(torch.zeros(4, 16, dtype=torch.uint8), torch.zeros(4, 1, dtype=torch.uint8))
+
+
+def test_zipf_workload_realises_the_skew():
+    """The skewed-routing recipe gives what the workload promises: the hottest expert near 25%
+    of assignments and several experts under 16 rows (top-k on the generated logits)."""
+    import torch
+    from mxfp4_quantized_moe_b200 import inputs
+    wl = inputs.WORKLOADS["gpt-oss-20b-moe-zipf-T16384"]
+    lg = inputs.make_workload(wl, 0, with_dy=False)["logits"]
+    h = torch.bincount(torch.topk(lg, wl.k, dim=1).indices.flatten(), minlength=wl.E)
+    assert 0.22 <= float(h.max()) / float(h.sum()) <= 0.28
+    assert int((h < 16).sum()) >= 5 and int(h.min()) >= 1
