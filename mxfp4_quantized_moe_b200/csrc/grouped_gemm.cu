@@ -93,8 +93,8 @@ struct SmemLayout {
   static constexpr int w = tok + kStages * kTokBytes;            // 256-aligned (32B swizzle)
   static constexpr int bars = w + kWStages * kWBytes;
   static constexpr int misc = bars + 512;                        // tmem slot, abort flag
-  static constexpr int cw = misc + 64;                           // 8 warps x 2 x 32 scale words
-  static constexpr int tables = cw + kConvWarps * 2 * 32 * 4;    // off[257], tile_start[257]
+  static constexpr int cw = misc + 64;                           // 8 warps x 4 x 32 scale words
+  static constexpr int tables = cw + kConvWarps * 4 * 32 * 4;    // off[257], tile_start[257]
   static constexpr int sc = ((tables + 2 * 257 * 4) + 127) / 128 * 128;  // 2 scale buffers
 };
 static_assert(SmemLayout::w % 1024 == 0, "weight ring alignment");
@@ -367,122 +367,163 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (wg < 3) {
     // ================================ converters ====================================
     if (kRegsConv < kLaunchRegs) setmaxnreg_dec<kRegsConv>();
-    // Converter warp c (0..7) serves TMEM lane quarter q = warp % 4 and the k-steps whose
-    // running index g has parity c / 4; its partner warp takes the other parity.
+    // Converter warp c (0..7) serves TMEM lane quarter q = warp % 4.  A tile's k-steps are
+    // converted in pairs (2u, 2u+1), the pairs the MMA issuer waits for and issues together;
+    // the two warps of a quarter take alternate pairs (running pair index parity = c / 4).
     const int q = warp & 3;
     const int cidx = warp - 4;
     const int par = cidx >> 2;
-    uint32_t* cw = reinterpret_cast<uint32_t*>(smem + SmemLayout::cw) + cidx * 64;
+    // per-warp scale-factor words (transposed scales): f1 of k-steps 0/1, then f2 of 0/1
+    uint32_t* cw = reinterpret_cast<uint32_t*>(smem + SmemLayout::cw) + cidx * 128;
     const int r = 32 * q + lane;  // row of the 128-row weight tile
     // 32B-swizzled packed tile: the two 16-byte halves of row r swap when bit 2 of r is set
     const int swz = (r >> 2) & 1;
-    int g = 0;
+    const int npair = (nk + 1) >> 1;
+    int g = 0;   // running index of the current tile's first k-step
+    int it = 0;  // running pair index
     int lt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt, g += nk) {
       Tile tl;
       decode_tile(t, s_tstart, s_off, E, nfb, tl);
       const bool active = tl.feat0 + 32 * q < N;  // warp-uniform: N % 32 == 0
       const int sb = lt & 1;
       if (!mbar_wait(smem_u32(&bar->sc_full[sb]), (lt >> 1) & 1, err, 0x400, s_abort)) break;
       const uint8_t* scb = s_sc + sb * sc_bytes;
-      for (int ks = 0; ks < nk; ++ks, ++g) {
-        if ((g & 1) != par) continue;
-        const int s = g % kWStages;
-        if (!mbar_wait(smem_u32(&bar->w_full[s]), (g / kWStages) & 1, err, 0x401, s_abort)) {
-          ok = false;
-          break;
-        }
-        uint32_t qw[8];
-        {
-          const uint8_t* row = smem + SmemLayout::w + s * kWBytes + r * (kBK / 2);
-          const uint4 w0 = *reinterpret_cast<const uint4*>(row + (swz << 4));
-          const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((swz ^ 1) << 4));
-          qw[0] = w0.x; qw[1] = w0.y; qw[2] = w0.z; qw[3] = w0.w;
-          qw[4] = w1.x; qw[5] = w1.y; qw[6] = w1.z; qw[7] = w1.w;
-        }
+      for (int u = 0; u < npair; ++u, ++it) {
+        if ((it & 1) != par) continue;
+        const int ks0 = 2 * u;
+        const bool two = ks0 + 1 < nk;
+        const int ga = g + ks0;  // running index of the pair's first k-step
         // scale factors: f1 (and f2 when some scale is above 128), as bf16x2 words
-        uint32_t f1a = 0, f1b = 0, f2a = 0x3F803F80u, f2b = 0x3F803F80u;
+        // (per row, forward: the pair's four 32-element blocks; the rare second factor is
+        // re-derived from the scale bytes where it is needed)
+        uint32_t f1[4];
         bool slow;
         if (!COLT) {
-          const uint32_t sA = active ? scb[r * kb32 + 2 * ks] : 127u;
-          const uint32_t sB = (active && 2 * ks + 1 < kb32) ? scb[r * kb32 + 2 * ks + 1] : 127u;
-          f1a = dup16(ue8m0_f1(sA));
-          f1b = dup16(ue8m0_f1(sB));
-          slow = __any_sync(kFull, (sA > 128u) | (sB > 128u));
-          if (slow) {
-            f2a = dup16(ue8m0_f2(sA));
-            f2b = dup16(ue8m0_f2(sB));
+          uint32_t mx = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int blk = 2 * ks0 + j;
+            const uint32_t sv = (active && blk < kb32) ? scb[r * kb32 + blk] : 127u;
+            mx = max(mx, sv);
+            f1[j] = dup16(ue8m0_f1(sv));
           }
+          slow = __any_sync(kFull, mx > 128u);
         } else {
-          // lane l computes the factors of K elements 2l, 2l+1 of this k-step; the warp
+          // lane l computes the factors of K elements 2l, 2l+1 of each k-step; the warp
           // shares them through shared memory (one scale row for all 32 lanes).
-          const int k0 = ks * kBK + 2 * lane;
-          uint32_t s0 = 127u, s1 = 127u;
-          if (active && k0 < K) {
-            s0 = scb[q * K + k0];
-            s1 = (k0 + 1 < K) ? scb[q * K + k0 + 1] : 127u;
+          uint32_t mx = 0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int k0 = (ks0 + h) * kBK + 2 * lane;
+            const uint32_t s0 = (active && k0 < K) ? scb[q * K + k0] : 127u;
+            const uint32_t s1 = (active && k0 + 1 < K) ? scb[q * K + k0 + 1] : 127u;
+            mx = max(mx, max(s0, s1));
+            cw[32 * h + lane] = ue8m0_f1(s0) | (ue8m0_f1(s1) << 16);
           }
-          slow = __any_sync(kFull, (s0 > 128u) | (s1 > 128u));
-          cw[lane] = ue8m0_f1(s0) | (ue8m0_f1(s1) << 16);
-          if (slow) cw[32 + lane] = ue8m0_f2(s0) | (ue8m0_f2(s1) << 16);
+          slow = __any_sync(kFull, mx > 128u);
+          if (slow) {  // rare: scales above 128 need the second factor
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int k0 = (ks0 + h) * kBK + 2 * lane;
+              const uint32_t s0 = (active && k0 < K) ? scb[q * K + k0] : 127u;
+              const uint32_t s1 = (active && k0 + 1 < K) ? scb[q * K + k0 + 1] : 127u;
+              cw[64 + 32 * h + lane] = ue8m0_f2(s0) | (ue8m0_f2(s1) << 16);
+            }
+          }
+          __syncwarp();  // cw written before any lane reads it
         }
-        // the packed bytes are in registers: release the weight stage
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar->w_empty[s]));
 
-        uint32_t out[32];
-        if (active) {
-          if (!COLT) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              uint32_t pt[4];
-              e2m1x8_to_bf16x2_pattern(qw[i], pt);
-              const uint32_t f1 = i < 4 ? f1a : f1b;
-#pragma unroll
-              for (int m = 0; m < 4; ++m) out[4 * i + m] = bmul2(pt[m], f1);
-            }
-            if (slow) {
-#pragma unroll
-              for (int m = 0; m < 32; ++m) out[m] = bmul2(out[m], m < 16 ? f2a : f2b);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              uint32_t pt[4];
-              e2m1x8_to_bf16x2_pattern(qw[i], pt);
-              const uint4 f = *reinterpret_cast<const uint4*>(cw + 4 * i);
-              out[4 * i + 0] = bmul2(pt[0], f.x);
-              out[4 * i + 1] = bmul2(pt[1], f.y);
-              out[4 * i + 2] = bmul2(pt[2], f.z);
-              out[4 * i + 3] = bmul2(pt[3], f.w);
-            }
-            if (slow) {
+        // each k-step: wait for its packed bytes, expand them to bf16 in registers, wait for
+        // its A stage to be free (the MMA consumed the k-step kStages earlier) and store it
+        const uint32_t lanes = (uint32_t)(32 * q) << 16;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !two) break;
+          const int s = (ga + h) % kWStages;
+          if (!mbar_wait(smem_u32(&bar->w_full[s]), ((ga + h) / kWStages) & 1, err, 0x401,
+                         s_abort)) {
+            ok = false;
+            break;
+          }
+          uint32_t qw[8];
+          {
+            const uint8_t* row = smem + SmemLayout::w + s * kWBytes + r * (kBK / 2);
+            const uint4 w0 = *reinterpret_cast<const uint4*>(row + (swz << 4));
+            const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((swz ^ 1) << 4));
+            qw[0] = w0.x; qw[1] = w0.y; qw[2] = w0.z; qw[3] = w0.w;
+            qw[4] = w1.x; qw[5] = w1.y; qw[6] = w1.z; qw[7] = w1.w;
+          }
+          uint32_t out[32];
+          if (active) {
+            if (!COLT) {
+              const uint32_t fa0 = h ? f1[2] : f1[0];
+              const uint32_t fa1 = h ? f1[3] : f1[1];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const uint4 f = *reinterpret_cast<const uint4*>(cw + 32 + 4 * i);
-                out[4 * i + 0] = bmul2(out[4 * i + 0], f.x);
-                out[4 * i + 1] = bmul2(out[4 * i + 1], f.y);
-                out[4 * i + 2] = bmul2(out[4 * i + 2], f.z);
-                out[4 * i + 3] = bmul2(out[4 * i + 3], f.w);
+                uint32_t pt[4];
+                e2m1x8_to_bf16x2_pattern(qw[i], pt);
+                const uint32_t fa = i < 4 ? fa0 : fa1;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) out[4 * i + m] = bmul2(pt[m], fa);
+              }
+              if (slow) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const int blk = 2 * (ks0 + h) + j;
+                  const uint32_t f2 =
+                      dup16(ue8m0_f2(blk < kb32 ? scb[r * kb32 + blk] : 127u));
+#pragma unroll
+                  for (int m = 16 * j; m < 16 * j + 16; ++m) out[m] = bmul2(out[m], f2);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                uint32_t pt[4];
+                e2m1x8_to_bf16x2_pattern(qw[i], pt);
+                const uint4 f = *reinterpret_cast<const uint4*>(cw + 32 * h + 4 * i);
+                out[4 * i + 0] = bmul2(pt[0], f.x);
+                out[4 * i + 1] = bmul2(pt[1], f.y);
+                out[4 * i + 2] = bmul2(pt[2], f.z);
+                out[4 * i + 3] = bmul2(pt[3], f.w);
+              }
+              if (slow) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const uint4 f = *reinterpret_cast<const uint4*>(cw + 64 + 32 * h + 4 * i);
+                  out[4 * i + 0] = bmul2(out[4 * i + 0], f.x);
+                  out[4 * i + 1] = bmul2(out[4 * i + 1], f.y);
+                  out[4 * i + 2] = bmul2(out[4 * i + 2], f.z);
+                  out[4 * i + 3] = bmul2(out[4 * i + 3], f.w);
+                }
               }
             }
           }
+          const int sa = (ga + h) % kStages;
+          if (!mbar_wait(smem_u32(&bar->empty[sa]), (((ga + h) / kStages) & 1) ^ 1, err, 0x402,
+                         s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (active) tmem_st32(tmem + lanes + kACol0 + sa * (kBK / 2), out);
         }
-        const int sa = g % kStages;
-        if (!mbar_wait(smem_u32(&bar->empty[sa]), ((g / kStages) & 1) ^ 1, err, 0x402,
-                       s_abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (active) {
-          tmem_st32(tmem + ((uint32_t)(32 * q) << 16) + kACol0 + sa * (kBK / 2), out);
-          tmem_wait_st();
-        }
+        if (!ok) break;
+        if (active) tmem_wait_st();
         tc_fence_before();
-        __syncwarp();  // also orders this k-step's reads of cw before the next writes
-        if (lane == 0) mbar_arrive(smem_u32(&bar->full[sa]));
+        // packed bytes consumed and A stages written: release the weight stages and publish
+        // the A stages (this also orders the pair's reads of cw before the next pair's writes)
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&bar->w_empty[ga % kWStages]));
+          mbar_arrive(smem_u32(&bar->full[ga % kStages]));
+          if (two) {
+            mbar_arrive(smem_u32(&bar->w_empty[(ga + 1) % kWStages]));
+            mbar_arrive(smem_u32(&bar->full[(ga + 1) % kStages]));
+          }
+        }
       }
       if (!ok) break;
       __syncwarp();
