@@ -119,6 +119,7 @@ def oracle_sample(wl, seed, n_tokens, inp=None):
         inp = inputs.make_workload(wl, seed)
     sel = np.arange(min(n_tokens, wl.T))
     n = inputs.as_numpy(inp, sel)
+    n["W"]["_dequant_cache"] = {}  # forward and backward of this sample share each expert's dequant
     t0 = time.perf_counter()
     f = O.moe_forward(n["x"], n["logits"], n["W"], wl.k)
     O.moe_backward(n["dy"], f, n["W"])
