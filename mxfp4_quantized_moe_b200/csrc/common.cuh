@@ -88,6 +88,23 @@ MOE_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const DevErr& err, int whe
   }
 }
 
+// Bounded wait that yields the issue slot between probes (for waits off the critical path).
+MOE_DEV bool mbar_wait_sleep(uint32_t bar, uint32_t parity, const DevErr& err, int where,
+                             volatile int* abort, uint32_t ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort && *abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      err.set(MXFP4_MOE_ERR_DEVICE_TIMEOUT, where);
+      if (abort) *abort = 1;
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA ---------------
 MOE_DEV void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");

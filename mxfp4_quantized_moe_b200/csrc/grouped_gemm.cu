@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           Tile tl;
           decode_tile(t, s_tstart, s_off, E, nfb, tl);
           for (int ks = 0; ks < nk; ++ks) {
-            if (!mbar_wait(smem_u32(&bar->empty[s]), ph ^ 1, err, 0x201, s_abort)) { ok = false; break; }
+            if (!mbar_wait_sleep(smem_u32(&bar->empty[s]), ph ^ 1, err, 0x201, s_abort, 64)) { ok = false; break; }
             const uint32_t fb = smem_u32(&bar->full[s]);
             mbar_arrive_expect_tx(fb, kTokBytes);
             tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           decode_tile(t, s_tstart, s_off, E, nfb, tl);
           const int rows = min(kBM, N - tl.feat0);
           const int sb = lt & 1;
-          if (!mbar_wait(smem_u32(&bar->sc_empty[sb]), ((lt >> 1) & 1) ^ 1, err, 0x200, s_abort)) break;
+          if (!mbar_wait_sleep(smem_u32(&bar->sc_empty[sb]), ((lt >> 1) & 1) ^ 1, err, 0x200, s_abort, 128)) break;
           uint32_t bytes;
           const uint8_t* src;
           if (COLT) {
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load(smem_u32(s_sc + sb * sc_bytes), src, bytes, smem_u32(&bar->sc_full[sb]));
           ++sc_issued;
           for (int ks = 0; ks < nk; ++ks) {
-            if (!mbar_wait(smem_u32(&bar->w_empty[ws]), wph ^ 1, err, 0x202, s_abort)) { ok = false; break; }
+            if (!mbar_wait_sleep(smem_u32(&bar->w_empty[ws]), wph ^ 1, err, 0x202, s_abort, 64)) { ok = false; break; }
             const uint32_t fb = smem_u32(&bar->w_full[ws]);
             mbar_arrive_expect_tx(fb, kWBytes);
             tma_load_2d(smem_u32(smem + SmemLayout::w + ws * kWBytes), &tmap_w, ks * (kBK / 2),
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode_tile(t, s_tstart, s_off, E, nfb, tl);
       const bool active = tl.feat0 + 32 * q < N;  // warp-uniform: N % 32 == 0
       const int sb = lt & 1;
-      if (!mbar_wait(smem_u32(&bar->sc_full[sb]), (lt >> 1) & 1, err, 0x400, s_abort)) break;
+      if (!mbar_wait_sleep(smem_u32(&bar->sc_full[sb]), (lt >> 1) & 1, err, 0x400, s_abort, 64)) break;
       const uint8_t* scb = s_sc + sb * sc_bytes;
       for (int u = 0; u < npair; ++u, ++it) {
         if ((it & 1) != par) continue;
@@ -442,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < 2; ++h) {
           if (h == 1 && !two) break;
           const int s = (ga + h) % kWStages;
-          if (!mbar_wait(smem_u32(&bar->w_full[s]), ((ga + h) / kWStages) & 1, err, 0x401,
-                         s_abort)) {
+          if (!mbar_wait_sleep(smem_u32(&bar->w_full[s]), ((ga + h) / kWStages) & 1, err, 0x401,
+                         s_abort, 32)) {
             ok = false;
             break;
           }
@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           anext[j] = __ldg(p.act + o);
         }
       }
-      if (!mbar_wait(smem_u32(&bar->acc_full[acc]), (lt >> 1) & 1, err, 0x500, s_abort)) break;
+      if (!mbar_wait_sleep(smem_u32(&bar->acc_full[acc]), (lt >> 1) & 1, err, 0x500, s_abort, 256)) break;
       tc_fence_after();
       float bias_f = 0.f;
       if ((EPI == kEpiGateUp || EPI == kEpiDown) && active)
