@@ -61,7 +61,10 @@ def peaks():
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a grouped GEMM,
 # from an ncu capture of this bench's workload; summaries under profiles/.  An entry counts
 # only while the kernel's sources hash to `sources`: after any change it reads as null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("gemm_gate_up_glu", "gpt-oss-20b-moe-T8192"): {"bytes": (471.3 + 526.4) * 1e6, "sources": "0407a3d2ce0b964c"},
+    ("gemm_dx_scatter", "gpt-oss-20b-moe-T8192"): {"bytes": (662.2 + 174.9) * 1e6, "sources": "0407a3d2ce0b964c"},
+}
 KERNEL_SOURCES = ("mxfp4_quantized_moe_b200/csrc/grouped_gemm.cu",
                   "mxfp4_quantized_moe_b200/csrc/common.cuh",
                   "mxfp4_quantized_moe_b200/csrc/kernels.h")
