@@ -188,6 +188,20 @@ MXFP4_MOE_API int mxfp4_moe_dequantize(const uint8_t* blocks, const uint8_t* sca
  * if the stream reported an error.  `where` (may be NULL) receives the device-side tag. */
 MXFP4_MOE_API int mxfp4_moe_check(void* ws, void* stream, int32_t* where);
 
+/* Self-test of failure detection (a diagnostic with no counterpart in the pages).  Enqueues one
+ * small kernel on `stream` whose two device-side waits are on barriers that nothing ever
+ * completes.  The first wait runs out after the library's one-second limit: it records
+ * MXFP4_MOE_ERR_DEVICE_TIMEOUT with tag 0xF00 in the error word at the start of `ws` and
+ * raises the kernel's abort flag; the second wait (started half a second later) must leave
+ * through that flag and sets the 32-bit word at byte offset 8 of `ws` to 1; the kernel then
+ * frees its tensor memory and returns.  Nothing faults and the CUDA context stays usable.
+ *   ws: device memory, at least 16 bytes, 16-byte aligned, the first 16 bytes zero (a fresh
+ *       workspace qualifies); the caller owns it.
+ * Returns OK once enqueued; the outcome is read with mxfp4_moe_check(ws, ...), which then
+ * returns DEVICE_TIMEOUT with *where == 0xF00.  Takes about one second of device time.
+ * Errors: INVALID_ARG (null, short or misaligned ws), UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream);
+
 /* Per-kernel timing (diagnostics).  Between mxfp4_moe_profile_begin() and
  * mxfp4_moe_profile_end(), the library records a CUDA event pair on the launching stream around
  * every kernel it enqueues (host-side bookkeeping only; results are unchanged).

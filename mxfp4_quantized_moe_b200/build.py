@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmxfp4_moe.so")
 SOURCES = ["csrc/api.cu", "csrc/grouped_gemm.cu", "csrc/kernels_small.cu",
-           "csrc/forward_static.cu"]
+           "csrc/forward_static.cu", "csrc/selftest.cu"]
 DEPS = SOURCES + ["csrc/common.cuh", "csrc/kernels.h"]
 
 

@@ -5,6 +5,8 @@
 #include <cstring>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/mxfp4_moe.h"
 #include "kernels.h"
 
@@ -155,12 +157,14 @@ struct Timed {
   cudaStream_t st;
   cudaEvent_t a = nullptr;
   Timed(const char* n, cudaStream_t s) : name(n), st(s) {
+    nvtxRangePushA(n);  // one NVTX range per kernel launch (free when no tool is attached)
     if (prof().on) {
       a = prof().get();
       cudaEventRecord(a, st);
     }
   }
   ~Timed() {
+    nvtxRangePop();
     if (a) {
       cudaEvent_t b = prof().get();
       cudaEventRecord(b, st);
@@ -319,6 +323,15 @@ int mxfp4_moe_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t r
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MOE_LAUNCH("dequant", moe::launch_dequant(blocks, scales, rows, K, out, st));
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 16 || !aligned16(ws)) return MXFP4_MOE_ERR_INVALID_ARG;
+  const int rc = check_device(nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_LAUNCH("selftest_wait_timeout", moe::launch_wait_timeout_selftest(static_cast<int*>(ws), st));
   return MXFP4_MOE_OK;
 }
 

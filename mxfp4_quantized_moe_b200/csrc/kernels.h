@@ -60,6 +60,9 @@ cudaError_t launch_dequant(const uint8_t* blocks, const uint8_t* scales, int64_t
                            uint16_t* out, cudaStream_t st);
 cudaError_t launch_transpose_packed(const uint8_t* src, int E, int R, int C, uint8_t* dst,
                                     cudaStream_t st);
+// One CTA whose mbarrier waits nothing completes: exercises the bounded-wait path (tag 0xF00
+// in the error word after about one second) without any fault.
+cudaError_t launch_wait_timeout_selftest(int* err_word, cudaStream_t st);
 cudaError_t launch_transpose_scales(const uint8_t* src, int E, int R, int C, uint8_t* dst,
                                     cudaStream_t st);
 

@@ -137,6 +137,13 @@ def device_check(ws: torch.Tensor, stream=None) -> tuple[int, int]:
     return rc, where.value
 
 
+def selftest_wait_timeout(ws: torch.Tensor, stream=None) -> None:
+    """Enqueue the failure-detection self-test on `ws` (first 16 bytes zero); read the outcome
+    with device_check(ws): (MXFP4_MOE_ERR_DEVICE_TIMEOUT, 0xF00) after about one second."""
+    check(lib.mxfp4_moe_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(),
+                                               _stream(stream)), "mxfp4_moe_selftest_wait_timeout")
+
+
 def weights_to(inp: dict, device) -> dict:
     keys = ("gu_blocks", "gu_scales", "gu_bias", "dn_blocks", "dn_scales", "dn_bias")
     return {k: inp[k].to(device).contiguous() for k in keys}

@@ -125,3 +125,9 @@ def test_zipf_workload_realises_the_skew():
     h = torch.bincount(torch.topk(lg, wl.k, dim=1).indices.flatten(), minlength=wl.E)
     assert 0.22 <= float(h.max()) / float(h.sum()) <= 0.28
     assert int((h < 16).sum()) >= 5 and int(h.min()) >= 1
+
+
+def test_selftest_arguments_checked_before_device(L):
+    assert L.lib.mxfp4_moe_selftest_wait_timeout(None, 64, None) == L.ERR_INVALID_ARG
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
+    assert L.lib.mxfp4_moe_selftest_wait_timeout(p, 8, None) == L.ERR_INVALID_ARG
