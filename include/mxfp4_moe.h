@@ -175,6 +175,21 @@ MXFP4_MOE_API int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_
                              size_t ws_bytes, uint16_t* dx, float* d_topk_w, float* d_logits,
                              void* stream);
 
+/* Layout helper: stacked gate_up rows to the interleaved order the block expects.
+ * "Integrate finegrained kernels: SOTA performance and per-module quantization", commit on the
+ * gate|up row interleave: GPT-OSS ships gate_up with gate j at row 2j and up j at row 2j+1,
+ * checkpoints stored with the halves stacked ([all gates; all ups]) must be converted by the
+ * caller, and the bytes cannot be inspected to tell which order a tensor is in.
+ *   stacked_blocks uint8 [E][2I][H/2], stacked_scales uint8 [E][2I][H/32], stacked_bias bf16
+ *   [E][2I] with row j = gate j and row I + j = up j; the outputs (same shapes, caller-owned,
+ *   not overlapping the inputs) receive row 2j = gate j and row 2j + 1 = up j.  Bytes are
+ *   copied unchanged (no re-quantization).  Uses d->E, d->H, d->I only.  Packed pointers must
+ *   be 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_interleave_gate_up(const mxfp4_moe_dims* d, const uint8_t* stacked_blocks,
+                                 const uint8_t* stacked_scales, const uint16_t* stacked_bias,
+                                 uint8_t* blocks, uint8_t* scales, uint16_t* bias, void* stream);
+
 /* Standalone dequantization (diagnostics and tests): rows of packed MXFP4 -> bf16.
  *   blocks uint8 [rows][K/2], scales uint8 [rows][K/32], out bf16 [rows][K]; K multiple of 32.
  * out = bf16(E2M1(code) * 2^(s-127)), exact (the product is always representable in bf16 or

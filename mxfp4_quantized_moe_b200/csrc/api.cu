@@ -326,6 +326,23 @@ int mxfp4_moe_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t r
   return MXFP4_MOE_OK;
 }
 
+int mxfp4_moe_interleave_gate_up(const mxfp4_moe_dims* d, const uint8_t* stacked_blocks,
+                                 const uint8_t* stacked_scales, const uint16_t* stacked_bias,
+                                 uint8_t* blocks, uint8_t* scales, uint16_t* bias, void* stream) {
+  if (!d || !stacked_blocks || !stacked_scales || !stacked_bias || !blocks || !scales || !bias)
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  if (d->E < 1 || d->E > 256 || d->H < 32 || d->H % 32 || d->I < 32 || d->I % 32)
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  if (!aligned16(stacked_blocks) || !aligned16(blocks)) return MXFP4_MOE_ERR_INVALID_ARG;
+  const int rc = check_device(nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_LAUNCH("interleave_gate_up",
+             moe::launch_interleave_gate_up(stacked_blocks, stacked_scales, stacked_bias, d->E, d->I,
+                                            d->H, blocks, scales, bias, st));
+  return MXFP4_MOE_OK;
+}
+
 int mxfp4_moe_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < 16 || !aligned16(ws)) return MXFP4_MOE_ERR_INVALID_ARG;
   const int rc = check_device(nullptr);

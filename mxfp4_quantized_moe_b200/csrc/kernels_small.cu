@@ -347,6 +347,33 @@ cudaError_t launch_dequant(const uint8_t* blocks, const uint8_t* scales, int64_t
   return cudaGetLastError();
 }
 
+// Stacked gate_up rows (gate j at row j, up j at row I + j) to the interleaved order (gate j
+// at row 2j, up j at row 2j + 1): one block per output row copies its packed bytes (16 bytes
+// per thread step), its scale bytes and its bias.
+__global__ void interleave_rows_kernel(const uint8_t* __restrict__ sb, const uint8_t* __restrict__ ss,
+                                       const uint16_t* __restrict__ sbias, int I, int K,
+                                       uint8_t* __restrict__ db, uint8_t* __restrict__ ds,
+                                       uint16_t* __restrict__ dbias) {
+  const int e = blockIdx.y;
+  const int r = blockIdx.x;              // output row in [0, 2I)
+  const int src = (r & 1) ? I + (r >> 1) : (r >> 1);
+  const size_t orow = (size_t)e * 2 * I + r, irow = (size_t)e * 2 * I + src;
+  const int nb = K / 2, ns = K / 32;     // packed bytes and scales per row
+  const uint4* bi = reinterpret_cast<const uint4*>(sb + irow * nb);
+  uint4* bo = reinterpret_cast<uint4*>(db + orow * nb);
+  for (int i = threadIdx.x; i < nb / 16; i += blockDim.x) bo[i] = bi[i];
+  for (int i = threadIdx.x; i < ns; i += blockDim.x) ds[orow * ns + i] = ss[irow * ns + i];
+  if (threadIdx.x == 0) dbias[orow] = sbias[irow];
+}
+
+cudaError_t launch_interleave_gate_up(const uint8_t* sb, const uint8_t* ss, const uint16_t* sbias,
+                                      int E, int I, int K, uint8_t* db, uint8_t* ds,
+                                      uint16_t* dbias, cudaStream_t st) {
+  dim3 grid(2 * I, E);
+  interleave_rows_kernel<<<grid, 64, 0, st>>>(sb, ss, sbias, I, K, db, ds, dbias);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_transpose_packed(const uint8_t* src, int E, int R, int C, uint8_t* dst,
                                     cudaStream_t st) {
   dim3 grid(C / 32, R / 32, E);

@@ -137,6 +137,17 @@ def device_check(ws: torch.Tensor, stream=None) -> tuple[int, int]:
     return rc, where.value
 
 
+def interleave_gate_up(shape: MoeShape, blocks: torch.Tensor, scales: torch.Tensor,
+                       bias: torch.Tensor, stream=None):
+    """Stacked gate_up (rows [gates; ups]) -> interleaved (gate j at 2j, up j at 2j+1);
+    returns new (blocks, scales, bias) tensors."""
+    ob, os_, obias = torch.empty_like(blocks), torch.empty_like(scales), torch.empty_like(bias)
+    check(lib.mxfp4_moe_interleave_gate_up(ctypes.byref(shape.dims()), _ptr(blocks), _ptr(scales),
+                                           _ptr(bias), _ptr(ob), _ptr(os_), _ptr(obias),
+                                           _stream(stream)), "mxfp4_moe_interleave_gate_up")
+    return ob, os_, obias
+
+
 def selftest_wait_timeout(ws: torch.Tensor, stream=None) -> None:
     """Enqueue the failure-detection self-test on `ws` (first 16 bytes zero); read the outcome
     with device_check(ws): (MXFP4_MOE_ERR_DEVICE_TIMEOUT, 0xF00) after about one second."""

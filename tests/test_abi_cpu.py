@@ -131,3 +131,11 @@ def test_selftest_arguments_checked_before_device(L):
     assert L.lib.mxfp4_moe_selftest_wait_timeout(None, 64, None) == L.ERR_INVALID_ARG
     p = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
     assert L.lib.mxfp4_moe_selftest_wait_timeout(p, 8, None) == L.ERR_INVALID_ARG
+
+
+def test_interleave_helper_arguments_checked_before_device(L):
+    d = L.Dims(16, 256, 256, 4, 2, 1.702, 7.0)
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced
+    assert L.lib.mxfp4_moe_interleave_gate_up(ctypes.byref(d), None, p, p, p, p, p, None) == L.ERR_INVALID_ARG
+    bad = L.Dims(16, 250, 256, 4, 2, 1.702, 7.0)
+    assert L.lib.mxfp4_moe_interleave_gate_up(ctypes.byref(bad), p, p, p, p, p, p, None) == L.ERR_INVALID_ARG

@@ -247,3 +247,21 @@ def test_run_to_run_deterministic(moe):
         outs.append([t.clone() for t in (y, dx, dtw, dl)])
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+def test_interleave_helper_restores_the_shipped_row_order(moe):
+    """Layout helper: a stacked checkpoint ([gates; ups]) converts to exactly the interleaved
+    tensors the block expects (bytes, scales and bias copied unchanged)."""
+    T, H, I, E, k = 16, 256, 288, 3, 2
+    inp = inputs.make_layer(T, H, I, E, k, 17)
+
+    def stacked(t):
+        return torch.cat([t[:, 0::2], t[:, 1::2]], dim=1).contiguous()
+
+    shape = moe.MoeShape(T, H, I, E, k)
+    ob, os_, obias = moe.interleave_gate_up(shape, stacked(inp["gu_blocks"]).cuda(),
+                                            stacked(inp["gu_scales"]).cuda(),
+                                            stacked(inp["gu_bias"]).cuda())
+    assert torch.equal(ob.cpu(), inp["gu_blocks"])
+    assert torch.equal(os_.cpu(), inp["gu_scales"])
+    assert torch.equal(obias.cpu(), inp["gu_bias"])
