@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmxfp4_moe.so")
 SOURCES = ["csrc/api.cu", "csrc/grouped_gemm.cu", "csrc/kernels_small.cu",
            "csrc/forward_static.cu", "csrc/selftest.cu"]
-DEPS = SOURCES + ["csrc/common.cuh", "csrc/kernels.h"]
+DEPS = SOURCES + ["csrc/common.cuh", "csrc/kernels.h", "csrc/aux_kernels.h"]
 
 
 def nvcc() -> str:

@@ -9,6 +9,7 @@
 
 #include "../../include/mxfp4_moe.h"
 #include "kernels.h"
+#include "aux_kernels.h"
 
 namespace {
 

@@ -58,16 +58,8 @@ cudaError_t launch_router_backward(const int32_t* idx, const float* w, const flo
                                    int T, int E, int k, float* d_logits, cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
                            uint16_t* out, cudaStream_t st);
-// Stacked gate_up rows [gates; ups] -> interleaved rows (gate j at 2j, up j at 2j+1) for
-// packed bytes [E][2I][K/2], scales [E][2I][K/32] and bias [E][2I]; K = H.
-cudaError_t launch_interleave_gate_up(const uint8_t* sb, const uint8_t* ss, const uint16_t* sbias,
-                                      int E, int I, int K, uint8_t* db, uint8_t* ds,
-                                      uint16_t* dbias, cudaStream_t st);
 cudaError_t launch_transpose_packed(const uint8_t* src, int E, int R, int C, uint8_t* dst,
                                     cudaStream_t st);
-// One CTA whose mbarrier waits nothing completes: exercises the bounded-wait path (tag 0xF00
-// in the error word after about one second) without any fault.
-cudaError_t launch_wait_timeout_selftest(int* err_word, cudaStream_t st);
 cudaError_t launch_transpose_scales(const uint8_t* src, int E, int R, int C, uint8_t* dst,
                                     cudaStream_t st);
 

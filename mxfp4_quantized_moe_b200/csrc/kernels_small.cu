@@ -3,6 +3,7 @@
 // GEMMs live in grouped_gemm.cu.
 #include "common.cuh"
 #include "kernels.h"
+#include "aux_kernels.h"
 
 namespace moe {
 

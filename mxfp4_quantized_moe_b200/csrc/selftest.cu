@@ -14,6 +14,7 @@
 #include "../../include/mxfp4_moe.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "aux_kernels.h"
 
 namespace moe {
 
