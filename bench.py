@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--kernel-table", action="store_true", help="print the per-kernel table to stderr")
     return ap.parse_args()
 
@@ -295,6 +295,10 @@ def main():
     ms_max = replicas.max_over_ranks(ms, dev)
 
     # ---- end to end through the public API with host buffers ----------------------------
+    # Every step copies its inputs (x, logits, dY) from pinned host memory and its results
+    # (y, dX, d_w, d_logits) back.  Steps are pipelined the way a training or serving loop
+    # would run them: two device buffer slots, step i computing on one while the inputs of
+    # step i+1 travel in and the results of step i-1 travel out on their own streams.
     hx = inp["x"].pin_memory()
     hlg = inp["logits"].pin_memory()
     hdy = inp["dy"].pin_memory()
@@ -302,27 +306,55 @@ def main():
     hdx = torch.empty_like(hy).pin_memory()
     hdtw = torch.empty(wl.T, wl.k, dtype=torch.float32).pin_memory()
     hdl = torch.empty(wl.T, wl.E, dtype=torch.float32).pin_memory()
+    slots = [dict(x=x, lg=lg, dy=dy, y=y, dx=dx, dtw=dtw, dl=dl),
+             dict(x=torch.empty_like(x), lg=torch.empty_like(lg), dy=torch.empty_like(dy),
+                  y=torch.empty_like(y), dx=torch.empty_like(dx), dtw=torch.empty_like(dtw),
+                  dl=torch.empty_like(dl))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {name: [torch.cuda.Event() for _ in range(2)]
+          for name in ("ready_in", "used_in", "computed", "copied_out")}
+    launched = {name: [False, False] for name in ev}
 
-    def e2e_step():
-        x.copy_(hx, non_blocking=True)
-        lg.copy_(hlg, non_blocking=True)
-        dy.copy_(hdy, non_blocking=True)
-        step()
-        hy.copy_(y, non_blocking=True)
-        hdx.copy_(dx, non_blocking=True)
-        hdtw.copy_(dtw, non_blocking=True)
-        hdl.copy_(dl, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        sl = slots[b]
+        with torch.cuda.stream(s_in):
+            if launched["used_in"][b]:
+                s_in.wait_event(ev["used_in"][b])
+            sl["x"].copy_(hx, non_blocking=True)
+            sl["lg"].copy_(hlg, non_blocking=True)
+            sl["dy"].copy_(hdy, non_blocking=True)
+            ev["ready_in"][b].record(s_in)
+        stream.wait_event(ev["ready_in"][b])
+        if launched["copied_out"][b]:
+            stream.wait_event(ev["copied_out"][b])
+        moe.forward(shape, w, sl["x"], sl["lg"], ws, y=sl["y"], stream=stream)
+        moe.backward_input(shape, w, wt, sl["dy"], ws, dx=sl["dx"], d_topk_w=sl["dtw"],
+                           d_logits=sl["dl"], stream=stream)
+        ev["used_in"][b].record(stream)
+        ev["computed"][b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["computed"][b])
+            hy.copy_(sl["y"], non_blocking=True)
+            hdx.copy_(sl["dx"], non_blocking=True)
+            hdtw.copy_(sl["dtw"], non_blocking=True)
+            hdl.copy_(sl["dl"], non_blocking=True)
+            ev["copied_out"][b].record(s_out)
+        for name in ("used_in", "copied_out"):
+            launched[name][b] = True
 
-    e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(s_in)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    s1.record(s_out)
     torch.cuda.synchronize()
-    e2e_ms = replicas.max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_ms = replicas.max_over_ranks(s0.elapsed_time(s1), dev)
     h2d = sum(int(v.numel() * v.element_size()) for v in (hx, hlg, hdy))
     d2h = sum(int(v.numel() * v.element_size()) for v in (hy, hdx, hdtw, hdl))
 
