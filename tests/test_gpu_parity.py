@@ -188,6 +188,8 @@ def test_tiny_workload_full_parity(moe):
     (200, 128, 64, 4, 4, 6, {"scale_lo": 110, "scale_hi": 140}),  # k == E; scales above 2^1
     (450, 64, 96, 2, 1, 7, {}),                                # several token tiles per expert
     (130, 2880, 2880, 4, 2, 8, {}),                            # gpt-oss widths, few tokens
+    (96, 64, 64, 256, 8, 9, {}),                               # E = 256 (the maximum), mostly empty
+    (24, 64, 96, 32, 20, 10, {}),                              # k = 20 > 16 selected per token
 ])
 def test_edge_cases(moe, T, H, I, E, k, seed, kw):
     got, ref = run_block(moe, T, H, I, E, k, seed, **kw)
