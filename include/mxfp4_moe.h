@@ -35,7 +35,8 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller, row-major, densely packed,
  *    at least 16-byte aligned.  "bf16" buffers are uint16_t bit patterns.  The library never
  *    allocates or frees device memory and never synchronizes the stream, except
- *    mxfp4_moe_check.
+ *    mxfp4_moe_check and mxfp4_moe_profile_end (mxfp4_moe_forward_static works on a static
+ *    device array that exists while the library is loaded).
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Work is
  *    enqueued on it and the call returns; results are valid once the stream reaches them.
  *  - Return value: 0 on success, a negative MXFP4_MOE_ERR_* code otherwise.  Argument errors
@@ -86,8 +87,8 @@ typedef struct {
  *   dn_blocks  uint8 [E][H][I/2]   down rows, same packing along I.
  *   dn_scales  uint8 [E][H][I/32]
  *   dn_bias    bf16  [E][H]
- * Stacked [gate; up] checkpoints must be interleaved by the caller first; the bytes do not
- * tell the two orders apart. */
+ * Stacked [gate; up] checkpoints must be interleaved first (mxfp4_moe_interleave_gate_up
+ * does it); the bytes do not tell the two orders apart. */
 typedef struct {
   const uint8_t* gu_blocks;
   const uint8_t* gu_scales;
