@@ -190,6 +190,8 @@ def test_tiny_workload_full_parity(moe):
     (130, 2880, 2880, 4, 2, 8, {}),                            # gpt-oss widths, few tokens
     (96, 64, 64, 256, 8, 9, {}),                               # E = 256 (the maximum), mostly empty
     (24, 64, 96, 32, 20, 10, {}),                              # k = 20 > 16 selected per token
+    (40, 32, 32, 4, 2, 11, {}),                                # H = I = 32: half a k-step
+    (33, 32, 96, 3, 2, 12, {}),                                # H = 32 forward, K = 192 back
 ])
 def test_edge_cases(moe, T, H, I, E, k, seed, kw):
     got, ref = run_block(moe, T, H, I, E, k, seed, **kw)
