@@ -355,3 +355,28 @@ def test_pins_catch_planted_mistakes(monkeypatch, mistake):
                             lambda h, d, a=1.702, l=7.0, **kw: orig_b(h, d, a, l, **kw)[..., ::-1])
     with pytest.raises(AssertionError):
         _check_all_pins()
+
+
+# ---------------------------------------------------------------- shapes at random ---
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=12, deadline=None)
+@given(T=st.integers(1, 5), H=st.sampled_from([32, 64, 96]), I=st.sampled_from([32, 64]),
+       E=st.integers(1, 5), kk=st.integers(1, 5), seed=st.integers(0, 10_000))
+def test_oracle_matches_scalar_twin_on_random_shapes(T, H, I, E, kk, seed):
+    """The vectorised oracle and the scalar twin agree for shapes other than the fixed pins
+    (H != I, one expert, k = E, single tokens): catches a transposed or mis-sliced operand that
+    happens to be invisible at square shapes."""
+    k = min(kk, E)
+    inp = inputs.make_layer(T, H, I, E, k, seed)
+    n = inputs.as_numpy(inp)
+    f = O.moe_forward(n["x"], n["logits"], n["W"], k)
+    dX, dw, dl = O.moe_backward(n["dy"], f, n["W"])
+    tw = scalar_twin.forward_backward(n["x"].tolist(), n["logits"].tolist(), n["dy"].tolist(),
+                                      n["W"], k)
+    assert np.array_equal(f["idx"], np.array(tw["idx"]))
+    np.testing.assert_allclose(f["out"], tw["out"], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dX, tw["dX"], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dw, tw["d_w"], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dl, tw["d_logits"], rtol=1e-9, atol=1e-11)
