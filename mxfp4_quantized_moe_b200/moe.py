@@ -118,13 +118,17 @@ def backward_input(shape: MoeShape, w: dict, wt: torch.Tensor, dy: torch.Tensor,
     return dx, d_topk_w, d_logits
 
 
-def dequantize(blocks: torch.Tensor, scales: torch.Tensor, stream=None) -> torch.Tensor:
+def dequantize(blocks: torch.Tensor, scales: torch.Tensor, stream=None,
+               out: torch.Tensor | None = None) -> torch.Tensor:
     """bf16 [rows, K] from packed uint8 [rows, K/2] and UE8M0 scales [rows, K/32]."""
     rows = blocks.numel() // blocks.shape[-1]
     K = blocks.shape[-1] * 2
     if scales.numel() != rows * (K // 32):
         raise ValueError("scales do not match blocks")
-    out = torch.empty(*blocks.shape[:-1], K, dtype=torch.bfloat16, device=blocks.device)
+    if out is None:
+        out = torch.empty(*blocks.shape[:-1], K, dtype=torch.bfloat16, device=blocks.device)
+    elif out.numel() != rows * K or out.dtype != torch.bfloat16:
+        raise ValueError("out must be bf16 with rows * K elements")
     check(lib.mxfp4_moe_dequantize(_ptr(blocks), _ptr(scales), rows, K, _ptr(out),
                                    _stream(stream)), "mxfp4_moe_dequantize")
     return out
