@@ -228,29 +228,25 @@ __global__ void router_backward_kernel(const int32_t* __restrict__ idx,
   }
 }
 
-// One thread per 32-element MX block: 16 packed bytes + 1 scale -> 64 bytes of bf16.
+// One thread per 8 elements (one 32-bit word of codes, a quarter of an MX block): a warp reads
+// 128 contiguous bytes of codes and writes 512 contiguous bytes of bf16.
 __global__ void dequant_kernel(const uint8_t* __restrict__ blocks,
-                               const uint8_t* __restrict__ scales, int64_t nblocks,
+                               const uint8_t* __restrict__ scales, int64_t nwords,
                                uint16_t* __restrict__ out) {
-  const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= nblocks) return;
-  const uint4 q = __ldg(reinterpret_cast<const uint4*>(blocks) + b);
-  const uint32_t s = scales[b];
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= nwords) return;
+  const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(blocks) + t);
+  const uint32_t s = __ldg(scales + (t >> 2));
   const uint32_t f1 = dup16(ue8m0_f1(s)), f2 = dup16(ue8m0_f2(s));
-  const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-  uint4* o = reinterpret_cast<uint4*>(out) + b * 4;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t p[4];
-    e2m1x8_to_bf16x2_pattern(qw[i], p);
-    uint4 v;
-    v.x = bmul2(bmul2(p[0], f1), f2);
-    v.y = bmul2(bmul2(p[1], f1), f2);
-    v.z = bmul2(bmul2(p[2], f1), f2);
-    v.w = bmul2(bmul2(p[3], f1), f2);
-    if (s == 255u) v = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);  // quiet NaN
-    o[i] = v;
-  }
+  uint32_t p[4];
+  e2m1x8_to_bf16x2_pattern(q, p);
+  uint4 v;
+  v.x = bmul2(bmul2(p[0], f1), f2);
+  v.y = bmul2(bmul2(p[1], f1), f2);
+  v.z = bmul2(bmul2(p[2], f1), f2);
+  v.w = bmul2(bmul2(p[3], f1), f2);
+  if (s == 255u) v = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);  // quiet NaN
+  reinterpret_cast<uint4*>(out)[t] = v;
 }
 
 // Packed nibble transpose: src [E][R][C/2] (packed along C) -> dst [E][C][R/2] (packed
@@ -342,9 +338,9 @@ cudaError_t launch_router_backward(const int32_t* idx, const float* w, const flo
 
 cudaError_t launch_dequant(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
                            uint16_t* out, cudaStream_t st) {
-  const int64_t nb = rows * (K / 32);
-  if (nb == 0) return cudaSuccess;
-  dequant_kernel<<<(unsigned)((nb + 255) / 256), 256, 0, st>>>(blocks, scales, nb, out);
+  const int64_t nw = rows * (K / 8);  // 32-bit words of codes
+  if (nw == 0) return cudaSuccess;
+  dequant_kernel<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(blocks, scales, nw, out);
   return cudaGetLastError();
 }
 
