@@ -139,3 +139,17 @@ def test_interleave_helper_arguments_checked_before_device(L):
     assert L.lib.mxfp4_moe_interleave_gate_up(ctypes.byref(d), None, p, p, p, p, p, None) == L.ERR_INVALID_ARG
     bad = L.Dims(16, 250, 256, 4, 2, 1.702, 7.0)
     assert L.lib.mxfp4_moe_interleave_gate_up(ctypes.byref(bad), p, p, p, p, p, p, None) == L.ERR_INVALID_ARG
+
+
+def test_no_usable_device_is_an_error_not_a_crash(L):
+    """Valid arguments on a host without a B200: the call reports an error before enqueuing."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible: the fake pointers below would reach a launch")
+    d = L.Dims(64, 256, 256, 8, 2, 1.702, 7.0)
+    p = ctypes.c_void_p(1 << 20)
+    w = L.Weights(p, p, p, p, p, p)
+    rc, need = _ws(L, 64, 256, 256, 8, 2, 1.702, 7.0)
+    rc = L.lib.mxfp4_moe_forward(ctypes.byref(d), ctypes.byref(w), p, p, p, None, None, p, need,
+                                 None)
+    assert rc in (L.ERR_CUDA, L.ERR_UNSUPPORTED_DEVICE)

@@ -269,3 +269,42 @@ def test_interleave_helper_restores_the_shipped_row_order(moe):
     assert torch.equal(ob.cpu(), inp["gu_blocks"])
     assert torch.equal(os_.cpu(), inp["gu_scales"])
     assert torch.equal(obias.cpu(), inp["gu_bias"])
+
+
+def _ws_offsets(T, E, k):
+    """Offsets of the routing regions in the forward's workspace (the library's layout: each
+    region starts 256-byte aligned, in the order error word, histogram, offsets, idx, w, perm,
+    inv)."""
+    def up(v):
+        return (v + 255) // 256 * 256
+    A = T * k
+    o, out = 0, {}
+    for name, size in (("err", 16), ("hist", 4 * E), ("off", 4 * (E + 1)), ("idx", 4 * A),
+                       ("w", 4 * A), ("perm", 4 * A), ("inv", 4 * A)):
+        out[name] = o
+        o = up(o + size)
+    return out
+
+
+def test_permutation_is_the_stable_expert_sort(moe):
+    """K2 exactly: off is the prefix sum of the expert histogram, perm lists each expert's
+    (token, slot) assignments in slot order, and inv is its inverse."""
+    T, H, I, E, k = 300, 64, 64, 7, 3
+    inp = inputs.make_layer(T, H, I, E, k, 31)
+    shape = moe.MoeShape(T, H, I, E, k)
+    w = moe.weights_to(inp, "cuda")
+    ws = moe.alloc_workspace(shape)
+    moe.forward(shape, w, inp["x"].cuda(), inp["logits"].cuda(), ws)
+    assert moe.device_check(ws) == (0, 0)
+    o, A = _ws_offsets(T, E, k), T * k
+
+    def region(name, n):
+        return ws[o[name]:o[name] + 4 * n].cpu().view(torch.int32).numpy()
+
+    idx = O.route(inp["logits"].numpy().astype(np.float64), k)[0].reshape(-1)
+    assert np.array_equal(region("idx", A), idx)
+    hist = np.bincount(idx, minlength=E)
+    assert np.array_equal(region("off", E + 1), np.concatenate([[0], np.cumsum(hist)]))
+    perm = region("perm", A)
+    assert np.array_equal(perm, np.argsort(idx, kind="stable"))
+    assert np.array_equal(region("inv", A)[perm], np.arange(A))
