@@ -153,3 +153,19 @@ def test_no_usable_device_is_an_error_not_a_crash(L):
     rc = L.lib.mxfp4_moe_forward(ctypes.byref(d), ctypes.byref(w), p, p, p, None, None, p, need,
                                  None)
     assert rc in (L.ERR_CUDA, L.ERR_UNSUPPORTED_DEVICE)
+
+
+def test_binding_without_the_library_fails_loudly(tmp_path):
+    """No silent fallback: importing the binding without the built library raises ImportError."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "mxfp4_quantized_moe_b200")
+    dst = tmp_path / "mxfp4_quantized_moe_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "try:\n    import mxfp4_quantized_moe_b200.moe\nexcept ImportError as e:\n"
+            "    print('IMPORT_ERROR', e); sys.exit(3)\nprint('LOADED')") % str(tmp_path)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
+                       cwd=str(tmp_path))
+    assert r.returncode == 3 and "IMPORT_ERROR" in r.stdout, r.stdout + r.stderr
