@@ -331,3 +331,42 @@ def stack_backward(dY, recs, layers, alpha: float = 1.702, limit: float = 7.0):
         per[l] = (g, dX, d_w, d_logits)
         g = g + dX + d_logits @ np.asarray(layers[l]["w_r"], np.float64).T
     return g, per
+
+
+# --------------------------------------------------------------------------------------
+# MXFP8 (E4M3) activations: the split a block-scaled forward would feed the tensor cores.
+# Not used by the current GPU path; these functions state the reading such a path is held to.
+# --------------------------------------------------------------------------------------
+E4M3_MAX = 448.0  # exponent field 15 with mantissa 110 (mantissa 111 there is NaN)
+
+
+def round_e4m3(v) -> np.ndarray:
+    """Round to the nearest E4M3 value, ties to even (OCP MX v1.0 E4M3: 1 sign bit, 4 exponent
+    bits with bias 7, 3 mantissa bits; exponent field 0 is subnormal with spacing 2^-9).
+    Magnitudes above the largest finite value, 448, give NaN (the format has no infinity)."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))  # a = m * 2^ex, m in [0.5, 1)
+    lead = np.maximum(ex - 1, -6)               # binade of the leading bit; subnormals share -6
+    q = np.ldexp(1.0, lead - 3)                 # spacing: 3 mantissa bits
+    r = np.round(a / q) * q                     # a / q is exact; np.round ties to even
+    out = np.copysign(r, v)
+    return np.where(r > E4M3_MAX, np.nan, out)
+
+
+def mx_split(x, block: int = BLOCK):
+    """Split each `block`-element run of x (along the last axis) into two E4M3 parts with a
+    shared power-of-two scale: x = (hi + lo) * 2^S up to the rounding of lo, where 2^S is the
+    smallest power of two that brings the run's largest magnitude to at most 448,
+    hi = e4m3(x / 2^S) and lo = e4m3(x / 2^S - hi).  Returns (hi, lo, S) with S per run."""
+    x = np.asarray(x, dtype=np.float64)
+    shp = x.shape
+    xb = x.reshape(-1, block)
+    amax = np.abs(xb).max(axis=1)
+    m, ex = np.frexp(np.where(amax > 0, amax / E4M3_MAX, 1.0))
+    S = np.where(m == 0.5, ex - 1, ex)          # ceil(log2(amax / 448)), exactly
+    S = np.where(amax > 0, S, 0).astype(np.int64)
+    y = np.ldexp(xb, -S[:, None])
+    hi = round_e4m3(y)
+    lo = round_e4m3(y - hi)
+    return hi.reshape(shp), lo.reshape(shp), S

@@ -380,3 +380,32 @@ def test_oracle_matches_scalar_twin_on_random_shapes(T, H, I, E, kk, seed):
     np.testing.assert_allclose(dX, tw["dX"], rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(dw, tw["d_w"], rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(dl, tw["d_logits"], rtol=1e-9, atol=1e-11)
+
+
+# ---------------------------------------------------------------- E4M3 split -----------
+def test_round_e4m3_matches_torch_float8_exhaustively():
+    """Every bf16 value of magnitude up to 448 rounds to E4M3 exactly as torch's own cast."""
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    v = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float()
+    keep = torch.isfinite(v) & (v.abs() <= 448.0)
+    v = v[keep]
+    ref = v.to(torch.float8_e4m3fn).float().double().numpy()
+    got = O.round_e4m3(v.double().numpy())
+    assert np.array_equal(got, ref)
+    assert np.isnan(O.round_e4m3(np.array([470.0, -1e6]))).all()
+
+
+def test_mx_split_is_exact_near_the_block_maximum_and_bounded_below_it():
+    rng = np.random.default_rng(4)
+    x = torch.from_numpy(rng.standard_normal((256, 64)) * np.exp(rng.uniform(-8, 8, (256, 1))))
+    x = x.to(torch.bfloat16).double().numpy()  # bf16 activations
+    hi, lo, S = O.mx_split(x)
+    xb, hb, lb = x.reshape(-1, 32), hi.reshape(-1, 32), lo.reshape(-1, 32)
+    y = np.ldexp(xb, -S[:, None])
+    amax = np.abs(y).max(axis=1)
+    assert np.all((amax > 224.0) & (amax <= 448.0))            # the smallest fitting scale
+    resid = np.abs(y - hb - lb)
+    near = np.abs(y) >= amax[:, None] * 2.0 ** -9               # within 2^9 of the maximum
+    assert np.all(resid[near] == 0.0)
+    assert np.all(resid <= 2.0 ** -10)                          # half the subnormal spacing
+    assert near.mean() > 0.95
