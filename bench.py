@@ -223,6 +223,7 @@ def run_reference(args, rank):
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
                    "sample_tokens_per_step": n_tok},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "cpu_count": os.cpu_count(),
                          "sample": f"{n_tok} tokens of the {wl.name} batch per step (fwd+bwd)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -421,6 +422,7 @@ def main():
         n_tok = 64
         n, dt = oracle_sample(wl, args.seed, n_tok, inp)
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "cpu_count": os.cpu_count(), "torch_threads": torch.get_num_threads(),
                "sample": f"first {n} tokens of the {wl.name} batch, fwd+bwd, fp64 numpy "
                          f"({dt:.1f} s)"}
 
