@@ -142,18 +142,25 @@ MXFP4_MOE_API int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_wei
  * process whose device memory belongs to another framework's pool, or a latency-critical
  * serving loop that cannot pay for cudaMalloc's implicit device synchronization.
  * What it does: exactly mxfp4_moe_forward, with the workspace taken from a fixed array of
- * MXFP4_MOE_STATIC_SCRATCH_BYTES (64 MiB) that the library holds in device memory on every
- * GPU where this entry point has run (allocated when the library's code is loaded there, kept
- * until the process exits).  Arguments mean what they mean for mxfp4_moe_forward; the caller
- * still provides x, logits, y and the optional topk_idx / topk_w.  No cudaMalloc, cudaFree or
- * other allocating call is made.
- * First call on a device: it looks up the array's device address (cudaGetSymbolAddress) with
- * that device current and caches it, so make that first call before any stream capture.
+ * MXFP4_MOE_STATIC_SCRATCH_BYTES (64 MiB) that the library holds in device memory.  The array
+ * exists in every CUDA context that loads the library's module holding it: under the CUDA 12
+ * default of lazy module loading, on each device where this entry point has run; with
+ * CUDA_MODULE_LOADING=EAGER, on every device the library is used on.  It stays until the
+ * process exits (or the context is destroyed).  Arguments mean what they mean for
+ * mxfp4_moe_forward; the caller still provides x, logits, y and the optional topk_idx /
+ * topk_w.  No cudaMalloc, cudaFree or other allocating call is made.
+ * Set-up: the first call in a context looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it together with the context
+ * handle, so make that first call before any stream capture.  A cudaDeviceReset (or any other
+ * teardown of the context) reloads the module, possibly at another address; the next call
+ * notices the new context and looks the address up again, so after a reset the first call
+ * must again come before any capture.
  * Sharing: every call uses the same array and leaves its contents there for the next call; the
  * call clears what must start at zero.  Calls that overlap on the GPU (other streams, other
  * host threads) race on the array and must be serialized by the caller.  The saved state it
- * leaves is not usable by mxfp4_moe_backward_input, and device-side faults of this form are
- * not reported (use the workspace form and mxfp4_moe_check to diagnose).
+ * leaves is not usable by mxfp4_moe_backward_input.  Device-side faults (an expired bounded
+ * wait, an index check) are recorded in the array's error word: read them with
+ * mxfp4_moe_forward_static_check.
  * Errors: WORKSPACE_TOO_SMALL when mxfp4_moe_workspace_size(d) exceeds
  * MXFP4_MOE_STATIC_SCRATCH_BYTES (at H = I = 2880, k = 4 that is above 480 tokens);
  * otherwise as mxfp4_moe_forward. */
@@ -161,6 +168,13 @@ MXFP4_MOE_API int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_wei
 MXFP4_MOE_API int mxfp4_moe_forward_static(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w,
                                            const uint16_t* x, const float* logits, uint16_t* y,
                                            int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Companion of mxfp4_moe_forward_static (no counterpart in the source pages): synchronizes
+ * `stream`, then reads and clears the error word of the static array in the current context,
+ * like mxfp4_moe_check does for a workspace.  Returns 0, DEVICE_TIMEOUT or DEVICE_BOUNDS (from
+ * the device, with the tag in *where, which may be NULL), CUDA if the stream reported an error,
+ * UNSUPPORTED_DEVICE on a device other than sm_100.  Allocates nothing. */
+MXFP4_MOE_API int mxfp4_moe_forward_static_check(void* stream, int32_t* where);
 
 /* Input-gradient backward through the frozen quantized weights (no weight gradient).
  *   wt       the transposed copy from mxfp4_moe_transpose_weights for the same weights
@@ -190,6 +204,31 @@ MXFP4_MOE_API int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_
 MXFP4_MOE_API int mxfp4_moe_interleave_gate_up(const mxfp4_moe_dims* d, const uint8_t* stacked_blocks,
                                  const uint8_t* stacked_scales, const uint16_t* stacked_bias,
                                  uint8_t* blocks, uint8_t* scales, uint16_t* bias, void* stream);
+
+/* Grouped matmul over expert-sorted rows with MXFP4 weights dequantized on the fly: the
+ * product the block's GEMMs are built on, without their epilogues ("Integrate finegrained
+ * kernels: SOTA performance and per-module quantization", the experts' grouped GEMM over
+ * expert-sorted rows; "Add MXFP4 training support via a dequantize-on-the-fly fallback",
+ * section "What this does": weights dequantized on the fly, packed storage never modified).
+ * For every expert e and row r in [off[e], off[e+1]):
+ *     out[r][n] = bf16( sum_k x[r][k] * W_e[n][k] )   (fp32 accumulation)
+ *   off     int32 [E+1] DEVICE, off[0] = 0, non-decreasing, off[E] = A
+ *   x       bf16  [A][K]
+ *   transposed == 0: blocks uint8 [E][N][K/2], scales uint8 [E][N][K/32] (the stored layout:
+ *                    W_e[n][k] = E2M1(code) * 2^(s[e][n][k/32] - 127))
+ *   transposed == 1: blocks uint8 [E][N][K/2], scales uint8 [E][N/32][K] (the layout
+ *                    mxfp4_moe_transpose_weights writes: W_e[n][k] uses s[e][n/32][k])
+ *   out     bf16  [A][N]
+ *   err_word  device int32[4] or NULL: a device-side fault (an expired bounded wait) is
+ *             recorded there; read it with mxfp4_moe_check.
+ * N and K multiples of 32, 1 <= E <= 256.  Used to test the fused dequantizer bit for bit
+ * (one-hot rows of x pick single weights), and usable as a grouped expert projection.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_grouped_matmul(int32_t E, int32_t N, int32_t K, int32_t A,
+                                           const int32_t* off, const uint16_t* x,
+                                           const uint8_t* blocks, const uint8_t* scales,
+                                           int32_t transposed, uint16_t* out, int32_t* err_word,
+                                           void* stream);
 
 /* Standalone dequantization (diagnostics and tests): rows of packed MXFP4 -> bf16.
  *   blocks uint8 [rows][K/2], scales uint8 [rows][K/32], out bf16 [rows][K]; K multiple of 32.

@@ -51,8 +51,12 @@ SIGNATURES = {
                                          _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_moe_forward_static": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Weights),
                                                 _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mxfp4_moe_forward_static_check": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int32)]),
     "mxfp4_moe_backward_input": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Weights),
                                                 _vp, _sz, _vp, _vp, _sz, _vp, _vp, _vp, _vp]),
+    "mxfp4_moe_grouped_matmul": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                ctypes.c_int32, _vp, _vp, _vp, _vp, ctypes.c_int32,
+                                                _vp, _vp, _vp]),
     "mxfp4_moe_dequantize": (ctypes.c_int, [_vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp]),
     "mxfp4_moe_check": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "mxfp4_moe_selftest_wait_timeout": (ctypes.c_int, [_vp, ctypes.c_size_t, _vp]),

@@ -17,27 +17,28 @@ constexpr size_t kAlign = 256;
 size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-  size_t err, hist, off, idx, w, perm, inv, dgu, act, dh, rows, cbias, dwp, dw, total;
+  size_t err, off, idx, w, perm, inv, w_row, blk_hist, dgu, act, dh, rows, total;
 };
 
+// Workspace regions, each 256-byte aligned, in this order.  The forward leaves the routing
+// (idx, w, perm, inv, w_row), the GLU derivative factors (dgu) and the expert outputs y in
+// expert-sorted row order (rows) for the backward.
 WsLayout ws_layout(const mxfp4_moe_dims& d) {
   const size_t A = (size_t)d.T * d.k;
   WsLayout L{};
   size_t o = 0;
-  L.err = o;    o = up(o + 16);
-  L.hist = o;   o = up(o + 4ull * d.E);
-  L.off = o;    o = up(o + 4ull * (d.E + 1));
-  L.idx = o;    o = up(o + 4 * A);
-  L.w = o;      o = up(o + 4 * A);
-  L.perm = o;   o = up(o + 4 * A);
-  L.inv = o;    o = up(o + 4 * A);
-  L.dgu = o;    o = up(o + 4 * A * d.I);       // saved GLU derivative factors (bf16 pairs)
-  L.act = o;    o = up(o + 2 * A * d.I);       // saved act [A][I]
-  L.dh = o;     o = up(o + 2 * A * 2 * d.I);   // dH [A][2I] (backward scratch)
-  L.rows = o;   o = up(o + 2 * A * d.H);       // Xp/Yslot (fwd), dYp/dXslot (bwd)
-  L.cbias = o;  o = up(o + 4 * A);
-  L.dwp = o;    o = up(o + 4 * A * (d.I / 32));
-  L.dw = o;     o = up(o + 4 * A);
+  L.err = o;      o = up(o + 16);
+  L.off = o;      o = up(o + 4ull * (d.E + 1));
+  L.idx = o;      o = up(o + 4 * A);                 // expert of each slot t*k+j
+  L.w = o;        o = up(o + 4 * A);                 // routing weight of each slot
+  L.perm = o;     o = up(o + 4 * A);                 // sorted row -> slot
+  L.inv = o;      o = up(o + 4 * A);                 // slot -> sorted row
+  L.w_row = o;    o = up(o + 4 * A);                 // routing weight of each sorted row
+  L.blk_hist = o; o = up(o + 4ull * moe::route_blocks(d.T) * d.E);
+  L.dgu = o;      o = up(o + 4 * A * d.I);           // saved GLU derivative factors (bf16 pairs)
+  L.act = o;      o = up(o + 2 * A * d.I);           // act [A][I] (the down GEMM's input)
+  L.dh = o;       o = up(o + 2 * A * 2 * d.I);       // dH [A][2I] (backward scratch)
+  L.rows = o;     o = up(o + 2 * A * d.H);           // Xp -> y (fwd), dYp -> dX rows (bwd)
   L.total = o;
   return L;
 }
@@ -235,31 +236,32 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->k, A = T * k;
   int* err = at<int>(ws, L.err);
-  int32_t* hist = at<int32_t>(ws, L.hist);
   int32_t* off = at<int32_t>(ws, L.off);
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* wr = at<float>(ws, L.w);
   int32_t* perm = at<int32_t>(ws, L.perm);
   int32_t* inv = at<int32_t>(ws, L.inv);
+  float* w_row = at<float>(ws, L.w_row);
+  int32_t* blk_hist = at<int32_t>(ws, L.blk_hist);
   uint16_t* dgu = at<uint16_t>(ws, L.dgu);
   uint16_t* act = at<uint16_t>(ws, L.act);
   uint16_t* rows = at<uint16_t>(ws, L.rows);
 
-  MOE_TRY(cudaMemsetAsync(hist, 0, 4ull * E, st));
-  MOE_LAUNCH("router_topk", moe::launch_router_topk(logits, T, E, k, idx, wr, hist, topk_idx, topk_w, err, st));
-  MOE_LAUNCH("build_perm", moe::launch_build_perm(idx, A, E, hist, off, perm, inv, err, st));
-  MOE_LAUNCH("gather_x", moe::launch_gather_rows(x, H, k, perm, A, rows, off, E, nullptr, nullptr, st));
+  MOE_LAUNCH("router_topk", moe::launch_router_topk(logits, T, E, k, idx, wr, blk_hist, topk_idx, topk_w, st));
+  MOE_LAUNCH("build_perm", moe::launch_build_perm(idx, wr, T, E, k, blk_hist, off, perm, inv, w_row, err, st));
+  MOE_LAUNCH("gather_x", moe::launch_gather_rows(x, H, k, perm, A, rows, nullptr, st));
 
   moe::GemmArgs g{};
-  g.off = off; g.E = E; g.A = A; g.perm = perm; g.topk_w = wr; g.err = err;
+  g.off = off; g.E = E; g.A = A; g.err = err;
   g.alpha = d->glu_alpha; g.limit = d->glu_limit; g.mask_limit = bf16_mask_limit(d->glu_limit);
   // gate_up: h = Xp W_gu^T + b_gu; act = GLU(h) and the GLU derivative factors are saved
   g.scales = w->gu_scales; g.K = H; g.N = 2 * I; g.bias = w->gu_bias; g.out0 = dgu; g.out1 = act;
   MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, rows, w->gu_blocks, g, sms, st));
-  // down: Yslot[slot] = w_slot * (act W_d^T + b_d)
+  // down: y = act W_d^T + b_d per sorted row (kept for the backward's routing-weight gradient)
   g.scales = w->dn_scales; g.K = I; g.N = H; g.bias = w->dn_bias; g.out0 = rows; g.out1 = nullptr;
-  MOE_LAUNCH("gemm_down_scatter", moe::launch_grouped_gemm(moe::kEpiDown, false, act, w->dn_blocks, g, sms, st));
-  MOE_LAUNCH("combine_y", moe::launch_combine(rows, T, k, H, y, st));
+  MOE_LAUNCH("gemm_down", moe::launch_grouped_gemm(moe::kEpiDown, false, act, w->dn_blocks, g, sms, st));
+  // out_t = sum_j w_{t,j} y_{t,j}
+  MOE_LAUNCH("combine_y", moe::launch_combine(rows, inv, wr, T, k, H, y, st));
   return MXFP4_MOE_OK;
 }
 
@@ -288,30 +290,45 @@ int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* wr = at<float>(ws, L.w);
   int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  const float* w_row = at<float>(ws, L.w_row);
   const uint32_t* dgu = at<uint32_t>(ws, L.dgu);
-  const uint16_t* act = at<uint16_t>(ws, L.act);
   uint16_t* dh = at<uint16_t>(ws, L.dh);
-  float* dw = at<float>(ws, L.dw);
   uint16_t* rows = at<uint16_t>(ws, L.rows);
-  float* cbias = at<float>(ws, L.cbias);
-  float* dwp = at<float>(ws, L.dwp);
 
-  // dYp[row] = dY[t(row)], cbias[row] = <dY[t], b_d[e(row)]>
-  MOE_LAUNCH("gather_dy_bias_dot", moe::launch_gather_rows(dy, H, k, perm, A, rows, off, E, w->dn_bias, cbias, st));
+  // d_topk_w[slot] = <dY_t, y_r> with the forward's y_r read in place, then dYp[r] = dY[t(r)]
+  MOE_LAUNCH("gather_dy_dw", moe::launch_gather_rows(dy, H, k, perm, A, rows, d_topk_w, st));
   moe::GemmArgs g{};
-  g.off = off; g.E = E; g.A = A; g.perm = perm; g.topk_w = wr; g.err = err;
+  g.off = off; g.E = E; g.A = A; g.err = err;
   g.alpha = d->glu_alpha; g.limit = d->glu_limit;
-  // dZ = dYp W_d (contract over H); epilogue: GLU derivative -> dH, partial <dZ, act>
-  g.scales = at<uint8_t>(wtp, LT.dn_scales); g.K = H; g.N = I; g.out0 = dh; g.dgu = dgu; g.act = act;
-  g.dw_part = dwp;
+  // dZ = dYp W_d (contract over H); epilogue: dact = w dZ, dH = dact * saved GLU factors
+  g.scales = at<uint8_t>(wtp, LT.dn_scales); g.K = H; g.N = I; g.out0 = dh; g.dgu = dgu; g.w_row = w_row;
   MOE_LAUNCH("gemm_dact_glu_bwd", moe::launch_grouped_gemm(moe::kEpiDact, true, rows, at<uint8_t>(wtp, LT.dn_blocks), g, sms, st));
-  // dx = dH W_gu (contract over the 2I interleaved rows)
-  g.scales = at<uint8_t>(wtp, LT.gu_scales); g.K = 2 * I; g.N = H; g.out0 = rows; g.dgu = nullptr; g.act = nullptr;
-  g.dw_part = nullptr;
-  MOE_LAUNCH("gemm_dx_scatter", moe::launch_grouped_gemm(moe::kEpiDx, true, dh, at<uint8_t>(wtp, LT.gu_blocks), g, sms, st));
-  MOE_LAUNCH("combine_dx", moe::launch_combine(rows, T, k, H, dx, st));
-  MOE_LAUNCH("reduce_dw", moe::launch_reduce_dw(cbias, dwp, I / 32, A, perm, dw, d_topk_w, st));
+  // dx = dH W_gu (contract over the 2I interleaved rows), per sorted row
+  g.scales = at<uint8_t>(wtp, LT.gu_scales); g.K = 2 * I; g.N = H; g.out0 = rows; g.dgu = nullptr; g.w_row = nullptr;
+  MOE_LAUNCH("gemm_dx", moe::launch_grouped_gemm(moe::kEpiDx, true, dh, at<uint8_t>(wtp, LT.gu_blocks), g, sms, st));
+  MOE_LAUNCH("combine_dx", moe::launch_combine(rows, inv, nullptr, T, k, H, dx, st));
   MOE_LAUNCH("router_backward", moe::launch_router_backward(idx, wr, d_topk_w, T, E, k, d_logits, st));
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_grouped_matmul(int32_t E, int32_t N, int32_t K, int32_t A, const int32_t* off,
+                             const uint16_t* x, const uint8_t* blocks, const uint8_t* scales,
+                             int32_t transposed, uint16_t* out, int32_t* err_word, void* stream) {
+  if (E < 1 || E > 256 || N < 32 || N % 32 || K < 32 || K % 32 || A < 0 || !off || !x ||
+      !blocks || !scales || !out || !aligned16(x) || !aligned16(blocks) || !aligned16(scales) ||
+      !aligned16(out) || (transposed != 0 && transposed != 1))
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  if (moe::grouped_gemm_smem_bytes(K) > 232448) return MXFP4_MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  const int rc = check_device(&sms);
+  if (rc) return rc;
+  if (A == 0) return MXFP4_MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  moe::GemmArgs g{};
+  g.off = off; g.E = E; g.A = A; g.err = reinterpret_cast<int*>(err_word);
+  g.scales = scales; g.K = K; g.N = N; g.out0 = out;
+  MOE_LAUNCH("grouped_matmul", moe::launch_grouped_gemm(moe::kEpiDx, transposed != 0, x, blocks, g, sms, st));
   return MXFP4_MOE_OK;
 }
 

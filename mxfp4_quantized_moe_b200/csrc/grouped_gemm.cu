@@ -542,17 +542,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int acc = lt & 1;
       const int f = tl.feat0 + 32 * q + lane;  // output feature of this thread
       const bool active = tl.feat0 + 32 * q < N;
-      // dact: the saved GLU factors and act of the tile's first 32 rows are requested before
-      // the accumulator is ready; each chunk then requests the next chunk's while it computes
+      // dact: the saved GLU factors of the tile's first 32 rows are requested before the
+      // accumulator is ready; each chunk then requests the next chunk's while it computes
       uint32_t dnext[32];
-      uint16_t anext[32];
       if (EPI == kEpiDact && active) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const size_t o = (size_t)min(tl.row0 + j, p.A - 1) * N + f;
-          dnext[j] = __ldg(p.dgu + o);
-          anext[j] = __ldg(p.act + o);
-        }
+        for (int j = 0; j < 32; ++j)
+          dnext[j] = __ldg(p.dgu + (size_t)min(tl.row0 + j, p.A - 1) * N + f);
       }
       if (!mbar_wait_sleep(smem_u32(&bar->acc_full[acc]), (lt >> 1) & 1, err, 0x500, s_abort, 256)) break;
       tc_fence_after();
@@ -606,23 +602,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          int my_slot = 0;
-          float my_w = 0.f;
-          if (lane < ncol) {
-            my_slot = p.perm[rbase + lane];
-            if (EPI == kEpiDown || EPI == kEpiDact) my_w = p.topk_w[my_slot];
-          }
           if (EPI == kEpiDown || EPI == kEpiDx) {
             // Feature pairs (f, f+1) live in lanes (2m, 2m+1): after one swap the even lane
-            // holds both features of column j, the odd lane both of column j+1.
+            // holds both features of column j, the odd lane both of column j+1.  Rows are
+            // stored in expert-sorted order (down: y = act W_d^T + b_d, not yet weighted; the
+            // combine applies the routing weights).
             uint32_t ow[16];
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
               float v0 = __uint_as_float(r[2 * jj]);
               float v1 = __uint_as_float(r[2 * jj + 1]);
               if (EPI == kEpiDown) {
-                v0 = __shfl_sync(kFull, my_w, 2 * jj) * (v0 + bias_f);
-                v1 = __shfl_sync(kFull, my_w, 2 * jj + 1) * (v1 + bias_f);
+                v0 += bias_f;
+                v1 += bias_f;
               }
               const float recv = __shfl_xor_sync(kFull, odd ? v0 : v1, 1);
               ow[jj] = odd ? pack_bf16x2(recv, v1) : pack_bf16x2(v0, recv);
@@ -631,41 +623,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
               const int col = 2 * jj + (odd ? 1 : 0);
-              const int slot = __shfl_sync(kFull, my_slot, col);
-              if (col < ncol) orow[((size_t)slot * N + (f & ~1)) >> 1] = ow[jj];
+              if (col < ncol) orow[((size_t)(rbase + col) * N + (f & ~1)) >> 1] = ow[jj];
             }
           } else {  // kEpiDact
             // dZ = dY W_d for this row; dact = w dZ; dH = (dact * dact/dg, dact * dact/du)
-            // from the factors the forward saved; partial <dZ, act> for the routing gradient.
+            // from the factors the forward saved.
             const int I = N;
             uint32_t* dh = reinterpret_cast<uint32_t*>(p.out0);
+            const float my_w = (lane < ncol) ? p.w_row[rbase + lane] : 0.f;
             uint32_t dcur[32];
-            uint16_t acur[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              dcur[j] = dnext[j];
-              acur[j] = anext[j];
-            }
+            for (int j = 0; j < 32; ++j) dcur[j] = dnext[j];
             if (c0 + 32 < tl.n_valid) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const size_t o = (size_t)min(rbase + 32 + j, p.A - 1) * I + f;
-                dnext[j] = __ldg(p.dgu + o);
-                anext[j] = __ldg(p.act + o);
-              }
+              for (int j = 0; j < 32; ++j)
+                dnext[j] = __ldg(p.dgu + (size_t)min(rbase + 32 + j, p.A - 1) * I + f);
             }
-            float part[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float wr = __shfl_sync(kFull, my_w, j);
-              const float dz = __uint_as_float(r[j]);
-              part[j] = (j < ncol) ? dz * bf16_to_f(acur[j]) : 0.f;
-              const float dact = wr * dz;
+              const float dact = __shfl_sync(kFull, my_w, j) * __uint_as_float(r[j]);
               const uint32_t dh2 = pack_bf16x2(dact * bf16_lo(dcur[j]), dact * bf16_hi(dcur[j]));
               if (j < ncol) dh[(size_t)(rbase + j) * I + f] = dh2;
             }
-            const float sum = warp_transpose_reduce(part, lane);
-            if (lane < ncol) p.dw_part[(size_t)((tl.feat0 >> 5) + q) * p.A + rbase + lane] = sum;
           }
         }
       }
@@ -758,6 +737,8 @@ cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const uint16_t*
     case kEpiDown * 2 + 0: return launch_one<kEpiDown, false>(tt, tw, a, grid, smem, st);
     case kEpiDact * 2 + 1: return launch_one<kEpiDact, true>(tt, tw, a, grid, smem, st);
     case kEpiDx * 2 + 1: return launch_one<kEpiDx, true>(tt, tw, a, grid, smem, st);
+    // plain product over the stored rows (the grouped matmul entry point)
+    case kEpiDx * 2 + 0: return launch_one<kEpiDx, false>(tt, tw, a, grid, smem, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -21,13 +21,11 @@ struct GemmArgs {
   const int32_t* off;      // [E+1] start row of each expert in the expert-sorted order
   int E, K, N, A;          // experts, contraction length, output features, assignments
   const uint16_t* bias;    // bf16 [E][N]: gate_up bias (kEpiGateUp) or down bias (kEpiDown)
-  uint16_t* out0;          // dGU [A][I] (bf16x2) | Yslot [A][H] | dH [A][2I] | dXslot [A][H]
+  uint16_t* out0;          // dGU [A][I] (bf16x2) | Y [A][H] | dH [A][2I] | dX rows [A][H],
+                           // all in expert-sorted row order
   uint16_t* out1;          // act [A][I] (kEpiGateUp)
   const uint32_t* dgu;     // saved GLU derivative factors [A][I] bf16x2 (kEpiDact)
-  const uint16_t* act;     // saved act [A][I] bf16 (kEpiDact)
-  const int32_t* perm;     // [A] sorted row -> slot t*k+j
-  const float* topk_w;     // [A] routing weight per slot
-  float* dw_part;          // [N/32][A] partial <dZ, act> sums (kEpiDact)
+  const float* w_row;      // [A] routing weight of each expert-sorted row (kEpiDact)
   float alpha, limit;
   float mask_limit;        // largest fp32 x whose bf16 rounding is <= limit (clamp-mask test)
   int* err;
@@ -40,19 +38,32 @@ cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const uint16_t*
                                 cudaStream_t st);
 size_t grouped_gemm_smem_bytes(int K);
 
+// Tokens are routed in blocks of a fixed size; blk_hist holds route_blocks(T) x E counts.
+int route_blocks(int T);
+// top-k + softmax over the k selected logits; idx/w in slot order (t*k + j), per-block
+// expert histograms in blk_hist [route_blocks(T)][E]
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
-                               int32_t* hist, int32_t* user_idx, float* user_w, int* err,
+                               int32_t* blk_hist, int32_t* user_idx, float* user_w,
                                cudaStream_t st);
-cudaError_t launch_build_perm(const int32_t* idx, int A, int E, const int32_t* hist, int32_t* off,
-                              int32_t* perm, int32_t* inv, int* err, cudaStream_t st);
+// stable expert sort of the slots: off[E+1], perm[row] = slot, inv[slot] = row,
+// w_row[row] = w[slot]
+cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, int k,
+                              const int32_t* blk_hist, int32_t* off, int32_t* perm, int32_t* inv,
+                              float* w_row, int* err, cudaStream_t st);
+// dst[r] = src[perm[r] / k] for every expert-sorted row r.  With `dot_w` (the backward's
+// gather of dY), `dst` first holds the forward's expert outputs y in sorted order, which are
+// read in place: dot_w[perm[r]] = <src[perm[r] / k], y[r]> before the row is overwritten.
 cudaError_t launch_gather_rows(const uint16_t* src, int H, int k, const int32_t* perm, int A,
-                               uint16_t* dst, const int32_t* off, int E, const uint16_t* bias,
-                               float* dot_out, cudaStream_t st);
-cudaError_t launch_combine(const uint16_t* slots, int T, int k, int H, uint16_t* out,
-                           cudaStream_t st);
-// dw[r] = cbias[r] + sum_p dw_part[p][r]; d_topk_w[perm[r]] = dw[r]  (one thread per row)
-cudaError_t launch_reduce_dw(const float* cbias, const float* dw_part, int nparts, int A,
-                             const int32_t* perm, float* dw, float* d_topk_w, cudaStream_t st);
+                               uint16_t* dst, float* dot_w, cudaStream_t st);
+// Gather x into expert-sorted rows as two E4M3 parts with a UE8M0 scale per 32 elements
+// (hi, lo [A][H] bytes; sfb [A][sfb_stride] bytes, the scale + 6 that the block-scaled
+// gate_up GEMM applies).
+cudaError_t launch_gather_quant(const uint16_t* x, int H, int k, const int32_t* perm, int A,
+                                uint8_t* hi, uint8_t* lo, uint8_t* sfb, int sfb_stride,
+                                cudaStream_t st);
+// out[t] = sum_j w[t*k+j] * rows[inv[t*k+j]] in fp32, rounded to bf16 once (w == nullptr: 1).
+cudaError_t launch_combine(const uint16_t* rows, const int32_t* inv, const float* w, int T, int k,
+                           int H, uint16_t* out, cudaStream_t st);
 // d_logits from d_topk_w through the softmax over the k selected logits (one thread per token)
 cudaError_t launch_router_backward(const int32_t* idx, const float* w, const float* d_topk_w,
                                    int T, int E, int k, float* d_logits, cudaStream_t st);

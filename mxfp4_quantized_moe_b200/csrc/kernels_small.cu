@@ -1,6 +1,8 @@
 // Routing, permutation, gather/combine, routing backward, standalone dequant and the
 // one-time weight transpose.  All of these are memory- or latency-bound; the grouped
 // GEMMs live in grouped_gemm.cu.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "aux_kernels.h"
@@ -13,168 +15,320 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---------------------------------------------------------------------------------------
 // Router: top-k over the E logits of a token (largest first, equal logits -> lower expert
-// index), softmax over the k selected, expert histogram.  One thread per token.
+// index), softmax over the k selected, and this block's expert histogram.  One warp per
+// token: lane l holds logits l, l+32, ... (E <= 256); each of the k rounds is a lane-local
+// best followed by a five-step butterfly argmax.  A block covers kRouteTokens consecutive
+// tokens, so its assignments are the contiguous slots [b*kRouteTokens*k, ...) and its
+// histogram (written to blk_hist[b][E], no global atomics) lets the permutation kernel place
+// them without another pass over the routing.
 // Source: the top-k router of the eager expert loop ("Add MXFP4 training support via a
 // dequantize-on-the-fly fallback", section "What this does"); softmax over the k values.
 // ---------------------------------------------------------------------------------------
-__global__ void router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                   int32_t* __restrict__ idx, float* __restrict__ w,
-                                   int32_t* __restrict__ hist, int32_t* __restrict__ user_idx,
-                                   float* __restrict__ user_w) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  const float* row = logits + (size_t)t * E;
-  uint32_t taken[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // E <= 256
-  int sel[16];
-  float val[16];
-  float m0 = 0.f, zsum = 0.f;
-  for (int j = 0; j < k; ++j) {
-    int best = -1;
-    float bv = 0.f;
-    for (int e = 0; e < E; ++e) {
-      if (taken[e >> 5] & (1u << (e & 31))) continue;
-      const float v = __ldg(row + e);
-      if (best < 0 || v > bv) {
-        best = e;
-        bv = v;
-      }
-    }
-    taken[best >> 5] |= 1u << (best & 31);
-    if (j == 0) m0 = bv;
-    const float z = __expf(bv - m0);
-    zsum += z;
-    if (j < 16) {
-      sel[j] = best;
-      val[j] = z;
-    }
-    atomicAdd(hist + best, 1);
-    idx[(size_t)t * k + j] = best;
-    w[(size_t)t * k + j] = z;  // normalized below
-  }
-  const float inv = 1.f / zsum;
-  for (int j = 0; j < k; ++j) {
-    const float z = (j < 16) ? val[j] : w[(size_t)t * k + j];
-    const int e = (j < 16) ? sel[j] : idx[(size_t)t * k + j];
-    const float wj = z * inv;
-    w[(size_t)t * k + j] = wj;
-    if (user_idx) user_idx[(size_t)t * k + j] = e;
-    if (user_w) user_w[(size_t)t * k + j] = wj;
-  }
+constexpr int kRouteThreads = 256;
+constexpr int kRouteTokens = 128;  // tokens per router / permutation block
+
+__device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
 }
 
-// ---------------------------------------------------------------------------------------
-// Stable counting sort of the A = T*k slots by expert.  Block e owns expert e: it scans
-// the slots in order and gives each slot of expert e the next row of [off[e], off[e+1]).
-// perm[row] = slot, inv[slot] = row.  Block 0 also publishes off[0..E].
-// ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) build_perm_kernel(const int32_t* __restrict__ idx, int A,
-                                                          int E, const int32_t* __restrict__ hist,
-                                                          int32_t* __restrict__ off,
-                                                          int32_t* __restrict__ perm,
-                                                          int32_t* __restrict__ inv, int* err) {
-  __shared__ int s_base;
-  __shared__ int s_warp[32];
-  __shared__ int s_run;
-  const int e = blockIdx.x;
-  if (threadIdx.x == 0) {
-    int base = 0;
-    for (int i = 0; i < e; ++i) base += hist[i];
-    s_base = base;
-    s_run = 0;
-    if (e == 0) {
-      int acc = 0;
-      for (int i = 0; i < E; ++i) {
-        off[i] = acc;
-        acc += hist[i];
+__global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
+    float* __restrict__ w, int32_t* __restrict__ blk_hist, int32_t* __restrict__ user_idx,
+    float* __restrict__ user_w) {
+  __shared__ int s_hist[256];
+  for (int e = threadIdx.x; e < E; e += kRouteThreads) s_hist[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_end = min(T, (blockIdx.x + 1) * kRouteTokens);
+  for (int t = blockIdx.x * kRouteTokens + warp; t < t_end; t += kRouteThreads / 32) {
+    const float* row = logits + (size_t)t * E;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      const float x = (e < E) ? __ldg(row + e) : -INFINITY;
+      v[i] = (x != x) ? -INFINITY : x;  // a NaN logit is never preferred
+    }
+    uint32_t taken = 0;  // bit i: expert lane + 32 i already selected (or absent)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (lane + 32 * i >= E) taken |= 1u << i;
+    float m0 = 0.f, zsum = 0.f;
+    float zr[8];
+    int ir[8];
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7FFFFFFF;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (!(taken & (1u << i)) && beats(v[i], lane + 32 * i, bv, bi)) {
+          bv = v[i];
+          bi = lane + 32 * i;
+        }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(kFull, bv, o);
+        const int oi = __shfl_xor_sync(kFull, bi, o);
+        if (beats(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
       }
-      off[E] = acc;
-      if (acc != A) DevErr{err}.set(MXFP4_MOE_ERR_DEVICE_BOUNDS, 0x100);
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (j == 0) m0 = bv;
+      const float z = __expf(bv - m0);
+      zsum += z;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (i == (j >> 5) && lane == (j & 31)) {
+          zr[i] = z;
+          ir[i] = bi;
+        }
+      if (lane == 0) atomicAdd(&s_hist[bi], 1);
+    }
+    const float inv = 1.f / zsum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = 32 * i + lane;
+      if (j < k) {
+        const size_t o = (size_t)t * k + j;
+        const float wj = zr[i] * inv;
+        idx[o] = ir[i];
+        w[o] = wj;
+        if (user_idx) user_idx[o] = ir[i];
+        if (user_w) user_w[o] = wj;
+      }
     }
   }
   __syncthreads();
-  const int base = s_base;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  for (int c = 0; c < A; c += blockDim.x) {
-    const int slot = c + threadIdx.x;
-    const bool f = slot < A && idx[slot] == e;
-    const unsigned b = __ballot_sync(kFull, f);
-    if (lane == 0) s_warp[wid] = __popc(b);
-    __syncthreads();
-    if (wid == 0) {
-      const int v = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
-      int incl = v;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += y;
-      }
-      s_warp[lane] = incl - v;  // exclusive prefix over the block's warps
+  for (int e = threadIdx.x; e < E; e += kRouteThreads)
+    blk_hist[(size_t)blockIdx.x * E + e] = s_hist[e];
+}
+
+// ---------------------------------------------------------------------------------------
+// Stable counting sort of the A = T*k slots by expert, one block per router block.  Block b
+// sums the router blocks' histograms into (a) the expert offsets off[e] (an exclusive scan of
+// the totals) and (b) the number of expert-e slots in blocks before b; its own slots are then
+// ranked in slot order: each warp counts a contiguous share of them per expert (warp-level
+// match on the expert id), a scan over the warps gives each share's first row, and a second
+// pass assigns the rows.  perm[row] = slot, inv[slot] = row, w_row[row] = w[slot]; block 0
+// publishes off[0..E].
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kRouteThreads) build_perm_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ w, int A, int E, int k,
+    const int32_t* __restrict__ blk_hist, int nblk, int32_t* __restrict__ off,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, float* __restrict__ w_row, int* err) {
+  constexpr int kWarps = kRouteThreads / 32;
+  __shared__ int s_cnt[kWarps][256];
+  __shared__ int s_tot[256];
+  __shared__ int s_scan[kWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x;
+  // (a) + (b): thread e sums column e of the [nblk][E] histograms
+  int before = 0, total = 0;
+  const int e = threadIdx.x;
+  if (e < E) {
+    for (int bb = 0; bb < nblk; ++bb) {
+      const int c = __ldg(blk_hist + (size_t)bb * E + e);
+      total += c;
+      if (bb < b) before += c;
     }
-    __syncthreads();
-    const int pos = s_run + s_warp[wid] + __popc(b & ((1u << lane) - 1u));
-    if (f) {
-      const int row = base + pos;
+  }
+  // exclusive scan of the totals over experts (E <= 256 = one value per thread)
+  int incl = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_scan[warp] = incl;
+  __syncthreads();
+  int wbase = 0;
+  for (int i = 0; i < warp; ++i) wbase += s_scan[i];
+  const int off_e = wbase + incl - total;
+  if (e < E) s_tot[e] = off_e + before;  // first row of this block's expert-e slots
+  if (b == 0) {
+    if (e < E) off[e] = off_e;
+    if (e == E - 1) {
+      off[E] = off_e + total;
+      if (off_e + total != A) DevErr{err}.set(MXFP4_MOE_ERR_DEVICE_BOUNDS, 0x100);
+    }
+  }
+  // this block's slots, split into kWarps contiguous shares of whole 32-slot steps
+  const int s0 = b * kRouteTokens * k, s1 = min(A, s0 + kRouteTokens * k);
+  const int steps = (s1 - s0 + 31) / 32;
+  const int per = (steps + kWarps - 1) / kWarps;
+  const int w0 = s0 + 32 * min(steps, warp * per), w1 = min(s1, s0 + 32 * min(steps, (warp + 1) * per));
+  for (int i = lane; i < E; i += 32) s_cnt[warp][i] = 0;
+  __syncwarp();
+  for (int c = w0; c < w1; c += 32) {  // pass 1: per-warp counts
+    const int slot = c + lane;
+    const int ex = slot < w1 ? idx[slot] : -1;
+    const unsigned m = __match_any_sync(kFull, ex);
+    if (ex >= 0 && lane == 31 - __clz(m)) s_cnt[warp][ex] += __popc(m);
+    __syncwarp();
+  }
+  __syncthreads();
+  if (e < E) {  // scan over the warps' shares
+    int run = s_tot[e];
+    for (int i = 0; i < kWarps; ++i) {
+      const int c = s_cnt[i][e];
+      s_cnt[i][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int c = w0; c < w1; c += 32) {  // pass 2: rows in slot order
+    const int slot = c + lane;
+    const int ex = slot < w1 ? idx[slot] : -1;
+    const unsigned m = __match_any_sync(kFull, ex);
+    if (ex >= 0) {
+      const int row = s_cnt[warp][ex] + __popc(m & ((1u << lane) - 1u));
       if (row < A) {
         perm[row] = slot;
         inv[slot] = row;
+        w_row[row] = w[slot];
       } else {
         DevErr{err}.set(MXFP4_MOE_ERR_DEVICE_BOUNDS, 0x101);
       }
     }
-    __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) s_run = pos + (f ? 1 : 0);
-    __syncthreads();
+    __syncwarp();
+    if (ex >= 0 && lane == 31 - __clz(m)) s_cnt[warp][ex] += __popc(m);
+    __syncwarp();
   }
 }
 
 // ---------------------------------------------------------------------------------------
-// dst[row] = src[perm[row] / k] for every expert-sorted row (one warp per row, 16-byte
-// vectors).  With `bias`, also dot_out[row] = <src row, bias[e(row)]> in fp32, e(row) the
-// expert owning the row (the down-bias term of the routing-weight gradient).
+// dst[r] = src[perm[r] / k] for every expert-sorted row r (one warp per row, 16-byte
+// vectors).  With `dot_w` (the backward's gather of dY), the row of `dst` first holds the
+// forward's expert output y_r (unweighted, bias included), read in place before it is
+// overwritten: dot_w[perm[r]] = <dY_t, y_r> in fp32, the routing-weight gradient.  Each lane
+// reads a 16-byte chunk of y_r and then writes the same chunk, and no other lane or warp
+// touches that chunk, so reading and writing one buffer is safe.
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ int expert_of_row(const int32_t* off, int E, int row) {
-  int lo = 0, hi = E;  // off[lo] <= row < off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(off + mid) <= row) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ src, int H, int k,
-                                   const int32_t* __restrict__ perm, int A,
-                                   uint16_t* __restrict__ dst, const int32_t* __restrict__ off,
-                                   int E, const uint16_t* __restrict__ bias,
-                                   float* __restrict__ dot_out) {
+                                   const int32_t* __restrict__ perm, int A, uint16_t* dst,
+                                   float* __restrict__ dot_w) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= A) return;
+  const int row = warp;
+  const int slot = perm[row];
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(slot / k) * H);
+  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * H);
+  const int nv = H / 8;
+  float acc = 0.f;
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 v = __ldg(s + i);
+    if (dot_w) {
+      const uint4 y = d[i];
+      acc += bf16_lo(v.x) * bf16_lo(y.x) + bf16_hi(v.x) * bf16_hi(y.x);
+      acc += bf16_lo(v.y) * bf16_lo(y.y) + bf16_hi(v.y) * bf16_hi(y.y);
+      acc += bf16_lo(v.z) * bf16_lo(y.z) + bf16_hi(v.z) * bf16_hi(y.z);
+      acc += bf16_lo(v.w) * bf16_lo(y.w) + bf16_hi(v.w) * bf16_hi(y.w);
+    }
+    d[i] = v;
+  }
+  if (dot_w) {
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    if (lane == 0) dot_w[slot] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Gather with the split into two E4M3 parts that the block-scaled gate_up GEMM consumes.
+// For every expert-sorted row r (token t = perm[r] / k) and 32-element block b of x[t]:
+//   S  = the smallest integer with max|x_block| <= 448 * 2^S (clamped to [-126, 121]),
+//   hi = e4m3(x / 2^S), lo = e4m3(x / 2^S - hi)   (round to nearest even, exact residual),
+//   sfb[r][b] = S + 133: the UE8M0 scale the MMA applies to both parts, 2^(S + 6), where the
+//   extra 2^6 undoes the weights' E2M1 -> E4M3 re-encoding (value * 2^-6) in the GEMM.
+// x / 2^S has at most 8 significant bits; hi keeps the top 4 and lo the next 4 (the remainder
+// is exact in fp32), so hi + lo equals x / 2^S for every element within 2^9 of the block
+// maximum that stays above the E4M3 subnormal floor; smaller elements keep an absolute error
+// below 2^-10 * 2^S.  A block holding inf or NaN gets the NaN scale (255).  Bytes of sfb past
+// the row's H/32 blocks are zero.  One warp per row; a lane takes whole blocks (64 bytes of
+// x in, 32 bytes of hi and of lo out).
+// Source: "Integrate finegrained kernels: SOTA performance and per-module quantization", the
+// commits on the activation format and input recipe (MX activations with UE8M0 block scales
+// feeding block-scaled tensor-core GEMMs).
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float a_lo, float a_hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(a_hi), "f"(a_lo));
+  return d;
+}
+__device__ __forceinline__ void f32x2_from_e4m3x2(uint32_t v, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "h"((uint16_t)v));
+  __half2 hh = *reinterpret_cast<__half2*>(&h2);
+  lo = __low2float(hh);
+  hi = __high2float(hh);
+}
+
+__global__ void gather_quant_kernel(const uint16_t* __restrict__ x, int H, int k,
+                                    const int32_t* __restrict__ perm, int A,
+                                    uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
+                                    uint8_t* __restrict__ sfb, int sfb_stride) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= A) return;
   const int row = warp;
   const int t = perm[row] / k;
-  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)t * H);
-  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * H);
-  const int nv = H / 8;
-  float acc = 0.f;
-  const uint4* bv = nullptr;
-  if (bias) bv = reinterpret_cast<const uint4*>(bias + (size_t)expert_of_row(off, E, row) * H);
-  for (int i = lane; i < nv; i += 32) {
-    const uint4 v = __ldg(s + i);
-    d[i] = v;
-    if (bias) {
-      const uint4 b = __ldg(bv + i);
-      acc += bf16_lo(v.x) * bf16_lo(b.x) + bf16_hi(v.x) * bf16_hi(b.x);
-      acc += bf16_lo(v.y) * bf16_lo(b.y) + bf16_hi(v.y) * bf16_hi(b.y);
-      acc += bf16_lo(v.z) * bf16_lo(b.z) + bf16_hi(v.z) * bf16_hi(b.z);
-      acc += bf16_lo(v.w) * bf16_lo(b.w) + bf16_hi(v.w) * bf16_hi(b.w);
+  const int nb = H / 32;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+  for (int b = lane; b < sfb_stride; b += 32) {
+    if (b >= nb) {
+      sfb[(size_t)row * sfb_stride + b] = 0;
+      continue;
     }
-  }
-  if (bias) {
-    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-    if (lane == 0) dot_out[row] = acc;
+    uint32_t v[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 q = __ldg(src + 4 * b + i);
+      v[4 * i + 0] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
+    }
+    uint32_t amax = 0;  // largest bf16 magnitude pattern (ordered like the magnitudes)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = max(amax, max(v[i] & 0x7FFFu, (v[i] >> 16) & 0x7FFFu));
+    uint32_t hw[8], lw[8];
+    int sbyte;
+    if (amax >= 0x7F80u) {  // inf or NaN in the block
+      sbyte = 255;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hw[i] = lw[i] = 0;
+    } else {
+      const int E = (int)(amax >> 7), m7 = (int)(amax & 0x7F);
+      const int S = (E == 0) ? -126 : max(-126, E - 135 + (m7 > 0x60 ? 1 : 0));
+      sbyte = S + 133;
+      const float inv = __uint_as_float((uint32_t)(127 - S) << 23);  // 2^-S, exact
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // elements 4i .. 4i+3
+        const float y0 = bf16_lo(v[2 * i]) * inv, y1 = bf16_hi(v[2 * i]) * inv;
+        const float y2 = bf16_lo(v[2 * i + 1]) * inv, y3 = bf16_hi(v[2 * i + 1]) * inv;
+        const uint32_t h01 = e4m3x2_from_f32(y0, y1), h23 = e4m3x2_from_f32(y2, y3);
+        float g0, g1, g2, g3;
+        f32x2_from_e4m3x2(h01, g0, g1);
+        f32x2_from_e4m3x2(h23, g2, g3);
+        const uint32_t l01 = e4m3x2_from_f32(y0 - g0, y1 - g1), l23 = e4m3x2_from_f32(y2 - g2, y3 - g3);
+        hw[i] = h01 | (h23 << 16);
+        lw[i] = l01 | (l23 << 16);
+      }
+    }
+    uint4* dh = reinterpret_cast<uint4*>(hi + (size_t)row * H + 32 * b);
+    uint4* dl = reinterpret_cast<uint4*>(lo + (size_t)row * H + 32 * b);
+    dh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    dh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    dl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    dl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    sfb[(size_t)row * sfb_stride + b] = (uint8_t)sbyte;
   }
 }
 
-// out[t] = sum_j slots[t*k + j] in fp32, rounded to bf16 once.  8 bf16 per thread.
-__global__ void combine_kernel(const uint16_t* __restrict__ slots, int T, int k, int H,
+// out[t] = sum_j w[t*k+j] * rows[inv[t*k+j]] in fp32 (w == nullptr: weight 1), rounded to
+// bf16 once.  8 bf16 per thread.
+__global__ void combine_kernel(const uint16_t* __restrict__ rows, const int32_t* __restrict__ inv,
+                               const float* __restrict__ w, int T, int k, int H,
                                uint16_t* __restrict__ out) {
   const int nv = H / 8;
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -182,11 +336,13 @@ __global__ void combine_kernel(const uint16_t* __restrict__ slots, int T, int k,
   const int t = (int)(i / nv), c = (int)(i % nv);
   float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   for (int j = 0; j < k; ++j) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(slots + ((size_t)t * k + j) * H) + c);
-    a[0] += bf16_lo(v.x); a[1] += bf16_hi(v.x);
-    a[2] += bf16_lo(v.y); a[3] += bf16_hi(v.y);
-    a[4] += bf16_lo(v.z); a[5] += bf16_hi(v.z);
-    a[6] += bf16_lo(v.w); a[7] += bf16_hi(v.w);
+    const size_t slot = (size_t)t * k + j;
+    const float wj = w ? __ldg(w + slot) : 1.f;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(rows + (size_t)__ldg(inv + slot) * H) + c);
+    a[0] += wj * bf16_lo(v.x); a[1] += wj * bf16_hi(v.x);
+    a[2] += wj * bf16_lo(v.y); a[3] += wj * bf16_hi(v.y);
+    a[4] += wj * bf16_lo(v.z); a[5] += wj * bf16_hi(v.z);
+    a[6] += wj * bf16_lo(v.w); a[7] += wj * bf16_hi(v.w);
   }
   uint4 o;
   o.x = pack_bf16x2(a[0], a[1]);
@@ -194,20 +350,6 @@ __global__ void combine_kernel(const uint16_t* __restrict__ slots, int T, int k,
   o.z = pack_bf16x2(a[4], a[5]);
   o.w = pack_bf16x2(a[6], a[7]);
   reinterpret_cast<uint4*>(out + (size_t)t * H)[c] = o;
-}
-
-// Routing-weight gradient per expert-sorted row: dw[r] = <dY_t, b_d[e]> + sum of the GEMM's
-// per-32-feature partial <dZ_r, act_r>; written to its slot.  Reads of the [P][A] partials
-// are coalesced across threads (consecutive rows).
-__global__ void reduce_dw_kernel(const float* __restrict__ cbias, const float* __restrict__ dw_part,
-                                 int nparts, int A, const int32_t* __restrict__ perm,
-                                 float* __restrict__ dw, float* __restrict__ d_topk_w) {
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= A) return;
-  float v = cbias[r];
-  for (int q = 0; q < nparts; ++q) v += __ldg(dw_part + (size_t)q * A + r);
-  dw[r] = v;
-  d_topk_w[perm[r]] = v;
 }
 
 // d_logits through the softmax over the k selected logits:
@@ -291,41 +433,47 @@ __global__ void transpose_scales_kernel(const uint8_t* __restrict__ src, int R, 
 
 }  // namespace
 
+int route_blocks(int T) { return (T + kRouteTokens - 1) / kRouteTokens; }
+
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
-                               int32_t* hist, int32_t* user_idx, float* user_w, int* err,
+                               int32_t* blk_hist, int32_t* user_idx, float* user_w,
                                cudaStream_t st) {
-  (void)err;
-  router_topk_kernel<<<(T + 127) / 128, 128, 0, st>>>(logits, T, E, k, idx, w, hist, user_idx,
-                                                      user_w);
+  router_topk_kernel<<<route_blocks(T), kRouteThreads, 0, st>>>(logits, T, E, k, idx, w, blk_hist,
+                                                                user_idx, user_w);
   return cudaGetLastError();
 }
 
-cudaError_t launch_build_perm(const int32_t* idx, int A, int E, const int32_t* hist, int32_t* off,
-                              int32_t* perm, int32_t* inv, int* err, cudaStream_t st) {
-  build_perm_kernel<<<E, 1024, 0, st>>>(idx, A, E, hist, off, perm, inv, err);
+cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, int k,
+                              const int32_t* blk_hist, int32_t* off, int32_t* perm, int32_t* inv,
+                              float* w_row, int* err, cudaStream_t st) {
+  const int nblk = route_blocks(T);
+  build_perm_kernel<<<nblk, kRouteThreads, 0, st>>>(idx, w, T * k, E, k, blk_hist, nblk, off, perm,
+                                                    inv, w_row, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const uint16_t* src, int H, int k, const int32_t* perm, int A,
-                               uint16_t* dst, const int32_t* off, int E, const uint16_t* bias,
-                               float* dot_out, cudaStream_t st) {
+                               uint16_t* dst, float* dot_w, cudaStream_t st) {
   const int threads = 256;
   const long long blocks = ((long long)A * 32 + threads - 1) / threads;
-  gather_rows_kernel<<<(unsigned)blocks, threads, 0, st>>>(src, H, k, perm, A, dst, off, E, bias,
-                                                           dot_out);
+  gather_rows_kernel<<<(unsigned)blocks, threads, 0, st>>>(src, H, k, perm, A, dst, dot_w);
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const uint16_t* slots, int T, int k, int H, uint16_t* out,
-                           cudaStream_t st) {
+cudaError_t launch_gather_quant(const uint16_t* x, int H, int k, const int32_t* perm, int A,
+                                uint8_t* hi, uint8_t* lo, uint8_t* sfb, int sfb_stride,
+                                cudaStream_t st) {
+  const int threads = 256;
+  const long long blocks = ((long long)A * 32 + threads - 1) / threads;
+  gather_quant_kernel<<<(unsigned)blocks, threads, 0, st>>>(x, H, k, perm, A, hi, lo, sfb,
+                                                            sfb_stride);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t* rows, const int32_t* inv, const float* w, int T, int k,
+                           int H, uint16_t* out, cudaStream_t st) {
   const size_t n = (size_t)T * (H / 8);
-  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(slots, T, k, H, out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_reduce_dw(const float* cbias, const float* dw_part, int nparts, int A,
-                             const int32_t* perm, float* dw, float* d_topk_w, cudaStream_t st) {
-  reduce_dw_kernel<<<(A + 255) / 256, 256, 0, st>>>(cbias, dw_part, nparts, A, perm, dw, d_topk_w);
+  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rows, inv, w, T, k, H, out);
   return cudaGetLastError();
 }
 

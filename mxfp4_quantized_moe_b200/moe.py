@@ -134,6 +134,21 @@ def dequantize(blocks: torch.Tensor, scales: torch.Tensor, stream=None,
     return out
 
 
+def grouped_matmul(off: torch.Tensor, x: torch.Tensor, blocks: torch.Tensor,
+                   scales: torch.Tensor, N: int, transposed: bool = False,
+                   err: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[r] = x[r] W_e^T for the rows r of expert e (off: int32 [E+1] on the device)."""
+    E = off.numel() - 1
+    A, K = x.shape
+    if x.dtype != torch.bfloat16 or off.dtype != torch.int32:
+        raise TypeError("x must be bf16 and off int32")
+    out = torch.empty(A, N, dtype=torch.bfloat16, device=x.device)
+    check(lib.mxfp4_moe_grouped_matmul(E, N, K, A, _ptr(off), _ptr(x), _ptr(blocks),
+                                       _ptr(scales), 1 if transposed else 0, _ptr(out),
+                                       _ptr(err), _stream(stream)), "mxfp4_moe_grouped_matmul")
+    return out
+
+
 def device_check(ws: torch.Tensor, stream=None) -> tuple[int, int]:
     """Synchronize and read (then clear) the device error word: (code, where)."""
     where = ctypes.c_int32(0)

@@ -66,9 +66,10 @@ def test_workspace_size_formula(L):
     rc, n = _ws(L, T, H, I, E, k, 1.702, 7.0)
     assert rc == 0
     A = T * k
-    # saved GLU factors (bf16x2) + saved act + dH + gathered rows + per-32-feature partials
-    big = A * (4 * I + 2 * I + 4 * I + 2 * H + 4 * (I // 32))
-    assert big <= n < big + 32 * A + 4 * 1024 * 1024
+    # saved GLU factors (bf16x2) + saved act + dH + rows (Xp / y / dYp / dX)
+    big = A * (4 * I + 2 * I + 4 * I + 2 * H)
+    # plus routing: idx, w, perm, inv, w_row (4 B each per assignment) and small tables
+    assert big + 20 * A <= n < big + 20 * A + 1024 * 1024
 
 
 @pytest.mark.parametrize("dims", [
@@ -91,6 +92,8 @@ def test_null_pointers_rejected_before_device(L):
                                         None, None, None, None)
     assert rc == L.ERR_INVALID_ARG
     rc = L.lib.mxfp4_moe_dequantize(None, None, 4, 64, None, None)
+    assert rc == L.ERR_INVALID_ARG
+    rc = L.lib.mxfp4_moe_grouped_matmul(2, 64, 64, 8, None, None, None, None, 0, None, None, None)
     assert rc == L.ERR_INVALID_ARG
     rc = L.lib.mxfp4_moe_dequantize(ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 48,
                                     ctypes.c_void_p(16), None)

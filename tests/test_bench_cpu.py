@@ -24,7 +24,7 @@ def test_algorithmic_work_and_bound():
     # FLOP: 2 * rows * N * K for each GEMM; the step is 12 A H I
     assert sum(f for f, _ in big.values()) == pytest.approx(12.0 * A * H * I)
     # packed gate_up weights alone are 0.5 + 1/32 bytes per element
-    assert big["gemm_dx_scatter"][1] >= E * 2 * I * H * (0.5 + 1 / 32)
+    assert big["gemm_dx"][1] >= E * 2 * I * H * (0.5 + 1 / 32)
     assert all(f / b > ridge for f, b in big.values())      # tensor-bound at T=8192
     assert all(f / b < ridge for f, b in small.values())    # weight streaming at T=256
 
@@ -51,3 +51,27 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["config"]["workload"] == "tiny-moe-T64-H256-E8-k2"
+
+
+def test_peak_choice_follows_region_length_and_clocks():
+    pk = {"bf16_tflops": 1644.9, "bf16_tflops_sustained": 1403.3, "hbm_gbs": 6550.0,
+          "source": "measured"}
+    boost = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}
+    capped = {"sm_mhz": 1680.0, "sm_max_mhz": 1965.0}
+    assert bench.choose_peak(pk, 0.08, boost)[:2] == (1644.9, "burst")
+    assert bench.choose_peak(pk, 0.08, capped)[:2] == (1403.3, "sustained")
+    assert bench.choose_peak(pk, 0.85, boost)[:2] == (1644.9, "burst")
+    assert bench.choose_peak(pk, 3.0, boost)[:2] == (1403.3, "sustained")
+    assert bench.choose_peak(pk, 0.08, None)[:2] == (1403.3, "sustained")
+
+
+def test_clock_sampler_keeps_only_samples_inside_the_region():
+    s = bench.ClockSampler(0)
+    s.thread = type("T", (), {"join": lambda self, timeout=None: None})()
+    s.source = "nvml"
+    s.rows = [(1.0, 1000.0, 1965.0, set()), (2.0, 1900.0, 1965.0, {"sw_power_cap"}),
+              (3.0, 1950.0, 1965.0, set()), (9.0, 500.0, 1965.0, set())]
+    s.mark(1.5, 3.5)
+    c = s.stop()
+    assert c["samples_in_timed_region"] == 2 and c["sm_mhz"] == 1925.0
+    assert c["reasons"] == ["sw_power_cap"] and c["sm_max_mhz"] == 1965.0

@@ -205,34 +205,69 @@ def test_expert_gradient_is_not_silent(moe):
     check_all(got, ref)
 
 
+def tile_boundary_tokens(logits, k, cap, seed, tile_rows=192):
+    """Tokens whose assignments sit on the first or last row of a grouped-GEMM token tile.
+
+    The GEMMs cut each expert's m expert-sorted rows into ceil(m / tile_rows) equal tiles of
+    a multiple of 16 rows (the last one possibly shorter); the rows at those cuts are where a
+    tile's TMA box starts or ends.  Returns at most `cap` of those tokens (seeded choice)."""
+    idx = O.route(np.asarray(logits, np.float64), k)[0].reshape(-1)
+    E = int(np.asarray(logits).shape[1])
+    hist = np.bincount(idx, minlength=E)
+    off = np.concatenate([[0], np.cumsum(hist)])
+    perm = np.argsort(idx, kind="stable")  # sorted row -> slot
+    rows = []
+    for e in range(E):
+        m = int(hist[e])
+        if m == 0:
+            continue
+        n = -(-m // tile_rows)
+        per = -(-m // n)
+        per = (per + 15) // 16 * 16
+        for start in range(0, m, per):
+            rows += [off[e] + start, off[e] + min(start + per, m) - 1]
+    toks = np.unique(perm[np.asarray(rows)] // k)
+    if toks.size > cap:
+        toks = np.sort(np.random.default_rng(seed).choice(toks, cap, replace=False))
+    return toks
+
+
 def test_gpt_oss_20b_full_size_sampled_tokens(moe):
-    """The benchmarked launch configuration (T=8192, H=I=2880, E=32, k=4), checked on a seeded
-    sample of tokens: every token is independent, so the oracle runs on the sample only."""
+    """The benchmarked launch configuration (T=8192, H=I=2880, E=32, k=4), checked on 1024
+    seeded random tokens plus tokens whose rows sit on token-tile boundaries: every token is
+    independent, so the oracle runs on the sample only.  Every token's output spans all 2880
+    features, the last 128-feature block (rows 2816..2879 of the weights) half full."""
     wl = inputs.WORKLOADS["gpt-oss-20b-moe-T8192"]
-    sel = np.sort(np.random.default_rng(0).choice(wl.T, 48, replace=False))
+    lg = inputs.make_workload(wl, 0, with_dy=False)["logits"].numpy()
+    rnd = np.random.default_rng(0).choice(wl.T, 1024, replace=False)
+    sel = np.union1d(rnd, tile_boundary_tokens(lg, wl.k, 256, 0))
     got, ref = run_block(moe, wl.T, wl.H, wl.I, wl.E, wl.k, seed=0, tokens=sel)
     check_all(got, ref)
 
 
 def test_zipf_skew_full_size_sampled_tokens(moe):
     """Skewed routing at T=16384 (hottest expert ~25% of assignments, eight experts under 16
-    rows): a seeded sample plus one token of each of the four coldest experts."""
+    rows): 256 seeded tokens, one token of each of the four coldest experts and tokens on
+    token-tile boundaries."""
     wl = inputs.WORKLOADS["gpt-oss-20b-moe-zipf-T16384"]
     lg = inputs.make_workload(wl, 0, with_dy=False)["logits"]
     idx = torch.topk(lg, wl.k, dim=1).indices
     cold = torch.bincount(idx.flatten(), minlength=wl.E).argsort()[:4]
     extra = [int((idx == e).any(dim=1).nonzero()[0]) for e in cold.tolist()]
-    rnd = np.random.default_rng(1).choice(wl.T, 24, replace=False).tolist()
-    sel = np.unique(np.asarray(rnd + extra))
+    rnd = np.random.default_rng(1).choice(wl.T, 256, replace=False).tolist()
+    sel = np.unique(np.concatenate([np.asarray(rnd + extra),
+                                    tile_boundary_tokens(lg.numpy(), wl.k, 64, 1)]))
     got, ref = run_block(moe, wl.T, wl.H, wl.I, wl.E, wl.k, seed=0, tokens=sel, zipf_s=wl.zipf_s)
     check_all(got, ref)
 
 
 def test_gpt_oss_120b_full_size_sampled_tokens(moe):
     """128 experts of ~512 rows (T=16384): many small expert groups, 1.69 GB of packed
-    weights streamed per pass."""
+    weights streamed per pass; 256 seeded tokens plus token-tile boundaries."""
     wl = inputs.WORKLOADS["gpt-oss-120b-moe-T16384"]
-    sel = np.sort(np.random.default_rng(2).choice(wl.T, 12, replace=False))
+    lg = inputs.make_workload(wl, 0, with_dy=False)["logits"].numpy()
+    rnd = np.random.default_rng(2).choice(wl.T, 256, replace=False)
+    sel = np.union1d(rnd, tile_boundary_tokens(lg, wl.k, 64, 2))
     got, ref = run_block(moe, wl.T, wl.H, wl.I, wl.E, wl.k, seed=0, tokens=sel)
     check_all(got, ref)
 
@@ -273,13 +308,12 @@ def test_interleave_helper_restores_the_shipped_row_order(moe):
 
 def _ws_offsets(T, E, k):
     """Offsets of the routing regions in the forward's workspace (the library's layout: each
-    region starts 256-byte aligned, in the order error word, histogram, offsets, idx, w, perm,
-    inv)."""
+    region starts 256-byte aligned, in the order error word, offsets, idx, w, perm, inv)."""
     def up(v):
         return (v + 255) // 256 * 256
     A = T * k
     o, out = 0, {}
-    for name, size in (("err", 16), ("hist", 4 * E), ("off", 4 * (E + 1)), ("idx", 4 * A),
+    for name, size in (("err", 16), ("off", 4 * (E + 1)), ("idx", 4 * A),
                        ("w", 4 * A), ("perm", 4 * A), ("inv", 4 * A)):
         out[name] = o
         o = up(o + size)

@@ -5,7 +5,7 @@ block's own inputs as the GPU saw them (x_l, logits_l and the upstream gradient 
 through the stack harness's forward and its recompute-per-block backward:
 
 * a small stack (4 blocks, T=64, H=I=256, E=8, k=2) on every token;
-* the full stack (24 gpt-oss-20b blocks, T=32768) on a sampled token, since each token's
+* the full stack (24 gpt-oss-20b blocks, T=32768) on 16 sampled tokens, since each token's
   path through the stack is independent of the other tokens.
 
 The stack output is not compared end to end with an fp64 chain: the caller rounds the
@@ -15,13 +15,17 @@ and clamp decisions downstream (an fp64 emulation of the bf16 stream alone drift
 router path, recompute order) is checked against the fp64 oracle stack on the CPU.
 """
 
+import multiprocessing
+import os
+from concurrent.futures import ProcessPoolExecutor
+
 import numpy as np
 import pytest
 import torch
 
 from mxfp4_quantized_moe_b200 import inputs, stack
-from oracle import mxfp4_oracle as O
 
+import oracle_pool
 from test_gpu_parity import assert_close, assert_d_logits_close
 
 pytestmark = pytest.mark.gpu
@@ -31,7 +35,7 @@ def _np(t):
     return t.detach().double().cpu().numpy()
 
 
-def _run_blockwise(wl, seed, sel):
+def _run_blockwise(wl, seed, sel, workers=1):
     """Runs the stack on the GPU, records the blocks' inputs and results for tokens `sel`,
     then checks every block against the oracle."""
     from mxfp4_quantized_moe_b200 import moe
@@ -55,17 +59,21 @@ def _run_blockwise(wl, seed, sel):
     del st, blocks, saved, out, g0
     torch.cuda.empty_cache()
 
-    for l in range(wl.layers):
-        inp = inputs.make_workload(wl, seed, layer=l, with_dy=False)
-        W = inputs.as_numpy(inp, [])["W"]
-        W["_dequant_cache"] = {}
-        f = O.moe_forward(_np(fw[l]["x"]), fw[l]["logits"].double().numpy(), W, wl.k)
-        assert_close(_np(fw[l]["y"]), f["out"], f"y[{l}]")
-        dX, d_w, d_logits = O.moe_backward(_np(bw[l]["g"]), f, W)
+    jobs = [(wl, seed, l, _np(fw[l]["x"]), fw[l]["logits"].double().numpy(), _np(bw[l]["g"]))
+            for l in range(wl.layers)]
+    if workers > 1:
+        # blocks are independent given their recorded inputs: fp64 oracle blocks in parallel
+        # worker processes (spawned: no CUDA state is inherited)
+        ctx = multiprocessing.get_context("spawn")
+        with ProcessPoolExecutor(max_workers=workers, mp_context=ctx) as ex:
+            refs = list(ex.map(oracle_pool.block, jobs))
+    else:
+        refs = [oracle_pool.block(j) for j in jobs]
+    for l, (out, dX, d_w, d_logits, w) in enumerate(refs):
+        assert_close(_np(fw[l]["y"]), out, f"y[{l}]")
         assert_close(_np(bw[l]["dx"]), dX, f"dx[{l}]")
         assert_close(_np(bw[l]["d_w"]), d_w, f"d_w[{l}]", np.float32)
-        assert_d_logits_close(_np(bw[l]["d_logits"]), d_logits, f["w"], d_w, f"d_logits[{l}]")
-        del inp, W
+        assert_d_logits_close(_np(bw[l]["d_logits"]), d_logits, w, d_w, f"d_logits[{l}]")
 
 
 def test_small_stack_blockwise_all_tokens():
@@ -73,6 +81,9 @@ def test_small_stack_blockwise_all_tokens():
     _run_blockwise(wl, 3, np.arange(wl.T))
 
 
-def test_stack24_full_size_blockwise_sampled_token():
+def test_stack24_full_size_blockwise_sampled_tokens():
+    """16 seeded tokens through all 24 blocks; each block's oracle touches most of its 32
+    experts, so the blocks are checked in parallel processes."""
     wl = inputs.WORKLOADS["gpt-oss-20b-moe-stack24-T32768"]
-    _run_blockwise(wl, 0, [int(np.random.default_rng(24).integers(wl.T))])
+    sel = np.sort(np.random.default_rng(24).choice(wl.T, 16, replace=False))
+    _run_blockwise(wl, 0, sel, workers=max(1, min(8, (os.cpu_count() or 2) // 2)))

@@ -65,6 +65,11 @@ def test_static_scratch_forward_matches_workspace_forward(T, H, I, E, k):
         assert torch.equal(ti, ti_ref), f"call {call}: routing differs"
         np.testing.assert_allclose(tw.cpu().numpy(), tw_ref.cpu().numpy(), rtol=2e-6, atol=1e-7)
         _close(y.float().cpu().numpy(), y_ref.float().cpu().numpy(), f"call {call}: y")
+        # the static array's error word: no device-side fault recorded
+        where = ctypes.c_int32(-1)
+        rc = L.lib.mxfp4_moe_forward_static_check(
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream), ctypes.byref(where))
+        assert (rc, where.value) == (0, 0), f"call {call}: device error {rc} at {where.value:#x}"
 
 
 def test_static_scratch_rejects_problems_larger_than_the_array():
