@@ -17,8 +17,12 @@ constexpr size_t kAlign = 256;
 size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-  size_t err, off, idx, w, perm, inv, w_row, blk_hist, dgu, act, dh, rows, total;
+  size_t err, off, idx, w, perm, inv, w_row, blk_hist, sfb, dgu, act, dh, rows, total;
 };
+
+// Row stride of the activation scales the block-scaled gate_up GEMM reads: one byte per
+// 32 elements of H, padded to whole k-steps (two blocks each) and to 16 bytes (bulk copies).
+int sfb_stride(int H) { return (2 * ((H + moe::kBK - 1) / moe::kBK) + 15) / 16 * 16; }
 
 // Workspace regions, each 256-byte aligned, in this order.  The forward leaves the routing
 // (idx, w, perm, inv, w_row), the GLU derivative factors (dgu) and the expert outputs y in
@@ -35,10 +39,12 @@ WsLayout ws_layout(const mxfp4_moe_dims& d) {
   L.inv = o;      o = up(o + 4 * A);                 // slot -> sorted row
   L.w_row = o;    o = up(o + 4 * A);                 // routing weight of each sorted row
   L.blk_hist = o; o = up(o + 4ull * moe::route_blocks(d.T) * d.E);
+  L.sfb = o;      o = up(o + A * sfb_stride(d.H));     // activation scales (gate_up)
   L.dgu = o;      o = up(o + 4 * A * d.I);           // saved GLU derivative factors (bf16 pairs)
   L.act = o;      o = up(o + 2 * A * d.I);           // act [A][I] (the down GEMM's input)
   L.dh = o;       o = up(o + 2 * A * 2 * d.I);       // dH [A][2I] (backward scratch)
-  L.rows = o;     o = up(o + 2 * A * d.H);           // Xp -> y (fwd), dYp -> dX rows (bwd)
+  L.rows = o;     o = up(o + 2 * A * d.H);           // E4M3 hi|lo of Xp -> y (fwd),
+                                                     // dYp -> dX rows (bwd)
   L.total = o;
   return L;
 }
@@ -68,7 +74,8 @@ int check_dims(const mxfp4_moe_dims* d) {
   if ((long long)d->T * d->k >= (1ll << 31)) return MXFP4_MOE_ERR_INVALID_ARG;
   if (!(d->glu_limit > 0.f) || !(d->glu_alpha == d->glu_alpha)) return MXFP4_MOE_ERR_INVALID_ARG;
   // the grouped GEMM keeps a tile's scales for the whole contraction in shared memory
-  if (moe::grouped_gemm_smem_bytes(d->H > 2 * d->I ? d->H : 2 * d->I) > 232448)
+  if (moe::grouped_gemm_smem_bytes(d->H > 2 * d->I ? d->H : 2 * d->I, 0) > 232448 ||
+      moe::grouped_gemm_smem_bytes(d->H, sfb_stride(d->H)) > 232448)
     return MXFP4_MOE_ERR_INVALID_ARG;
   return MXFP4_MOE_OK;
 }
@@ -249,14 +256,21 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
 
   MOE_LAUNCH("router_topk", moe::launch_router_topk(logits, T, E, k, idx, wr, blk_hist, topk_idx, topk_w, st));
   MOE_LAUNCH("build_perm", moe::launch_build_perm(idx, wr, T, E, k, blk_hist, off, perm, inv, w_row, err, st));
-  MOE_LAUNCH("gather_x", moe::launch_gather_rows(x, H, k, perm, A, rows, nullptr, st));
+  // Xp in expert-sorted order as two E4M3 parts (hi | lo in `rows`) with UE8M0 block scales
+  uint8_t* xhi = reinterpret_cast<uint8_t*>(rows);
+  uint8_t* xlo = xhi + (size_t)A * H;
+  uint8_t* sfb = at<uint8_t>(ws, L.sfb);
+  MOE_LAUNCH("gather_x_mx", moe::launch_gather_quant(x, H, k, perm, A, xhi, xlo, sfb, sfb_stride(H), st));
 
   moe::GemmArgs g{};
   g.off = off; g.E = E; g.A = A; g.err = err;
   g.alpha = d->glu_alpha; g.limit = d->glu_limit; g.mask_limit = bf16_mask_limit(d->glu_limit);
   // gate_up: h = Xp W_gu^T + b_gu; act = GLU(h) and the GLU derivative factors are saved
+  // (block-scaled: E2M1 weights against the E4M3 parts, fp32 accumulation)
   g.scales = w->gu_scales; g.K = H; g.N = 2 * I; g.bias = w->gu_bias; g.out0 = dgu; g.out1 = act;
-  MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, rows, w->gu_blocks, g, sms, st));
+  g.tok_lo = xlo; g.sfb = sfb; g.sfb_stride = sfb_stride(H);
+  MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, xhi, w->gu_blocks, g, sms, st));
+  g.tok_lo = nullptr; g.sfb = nullptr; g.sfb_stride = 0;
   // down: y = act W_d^T + b_d per sorted row (kept for the backward's routing-weight gradient)
   g.scales = w->dn_scales; g.K = I; g.N = H; g.bias = w->dn_bias; g.out0 = rows; g.out1 = nullptr;
   MOE_LAUNCH("gemm_down", moe::launch_grouped_gemm(moe::kEpiDown, false, act, w->dn_blocks, g, sms, st));
@@ -319,7 +333,7 @@ int mxfp4_moe_grouped_matmul(int32_t E, int32_t N, int32_t K, int32_t A, const i
       !blocks || !scales || !out || !aligned16(x) || !aligned16(blocks) || !aligned16(scales) ||
       !aligned16(out) || (transposed != 0 && transposed != 1))
     return MXFP4_MOE_ERR_INVALID_ARG;
-  if (moe::grouped_gemm_smem_bytes(K) > 232448) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (moe::grouped_gemm_smem_bytes(K, 0) > 232448) return MXFP4_MOE_ERR_INVALID_ARG;
   int sms = 0;
   const int rc = check_device(&sms);
   if (rc) return rc;

@@ -177,6 +177,29 @@ MOE_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+MOE_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+MOE_DEV void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+MOE_DEV void tmem_st1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
+MOE_DEV void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
 MOE_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -189,6 +212,40 @@ MOE_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr)
       : "memory");
+}
+
+// D[tmem] (+)= (A[tmem] x SFA) * (B[smem desc] x SFB); kind::mxf8f6f4 with one UE8M0 scale
+// per 32 elements of K on each side (scale_vec::1X), fp32 accumulate.  sfa/sfb are the TMEM
+// addresses of the scale-factor columns; which byte of them the MMA uses comes from the
+// instruction descriptor's scale-factor ids.
+MOE_DEV void mma_mxf8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], [%1], %2, %3, "
+      "[%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA with 64-byte
+// swizzle: rows of 64 bytes (64 E4M3 values), 8-row core groups 512 bytes apart.
+MOE_DEV uint64_t smem_desc_kmajor_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
+  d |= (uint64_t)1u << 16;                   // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(512u >> 4) << 32;           // stride byte offset: next 8-row group
+  d |= (uint64_t)1u << 46;                   // descriptor version (sm_100)
+  d |= (uint64_t)4u << 61;                   // 64-byte swizzle
+  return d;
+}
+// Instruction descriptor of the block-scaled MMA: A = E2M1 (format 5, one code per byte in
+// bits 5..2), B = E4M3 (format 0), UE8M0 scales, fp32 D, both K-major, M = 128, N = n; the
+// scale-factor ids pick byte `sfid` of each scale column.
+MOE_DEV uint32_t idesc_mxf4a_m128(int n, uint32_t sfid) {
+  return (sfid << 4) | (5u << 7) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) |
+         (sfid << 29);
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA with
@@ -253,6 +310,17 @@ MOE_DEV void e2m1x8_to_bf16x2_pattern(uint32_t q, uint32_t (&p)[4]) {
   p[1] = (prmt(ev, od, 0x9591u) * 0x1040u) & 0x81C081C0u;
   p[2] = (prmt(ev, od, 0xA6A2u) * 0x1040u) & 0x81C081C0u;
   p[3] = (prmt(ev, od, 0xB7B3u) * 0x1040u) & 0x81C081C0u;
+}
+
+// Eight packed E2M1 codes (byte i of q: element 2i in the low nibble, 2i+1 in the high one)
+// -> eight bytes in element order, each code in bits 5..2 of its byte: the 8-bit container
+// the block-scaled MMA reads E2M1 A operands from in tensor memory.  The codes are not
+// decoded; the MMA applies the E2M1 values and the UE8M0 scales itself.
+MOE_DEV void e2m1x8_to_containers(uint32_t q, uint32_t& lo4, uint32_t& hi4) {
+  const uint32_t ev = (q << 2) & 0x3C3C3C3Cu;  // elements 0, 2, 4, 6
+  const uint32_t od = (q >> 2) & 0x3C3C3C3Cu;  // elements 1, 3, 5, 7
+  lo4 = prmt(ev, od, 0x5140u);                 // elements 0, 1, 2, 3
+  hi4 = prmt(ev, od, 0x7362u);                 // elements 4, 5, 6, 7
 }
 
 // UE8M0 scale s -> two bf16 factors f1, f2 with pattern * f1 * f2 = value * 2^(s-127)

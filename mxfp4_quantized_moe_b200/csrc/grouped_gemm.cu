@@ -69,6 +69,15 @@ static_assert(128 * kRegsCtl + 2 * 128 * kRegsConv + 128 * kRegsEpi <= kThreads 
               "register split exceeds the block's launch allocation: setmaxnreg.inc would wait forever");
 static_assert(kRegsCtl % 8 == 0 && kRegsConv % 8 == 0 && kRegsEpi % 8 == 0, "setmaxnreg granularity");
 static_assert(kACol0 + kStages * (kBK / 2) <= kTmemCols, "TMEM budget");
+// Block-scaled variant (E2M1 weights in 8-bit containers against E4M3 tokens, UE8M0 scales):
+// A stages of 64 bytes (16 columns), then per stage the scale-factor columns of A (4) and of
+// the token tile (8, of which kBN/32 are used).
+constexpr int kAColsBS = kBK / 4;
+constexpr int kSfaCol0 = kACol0 + kStages * kAColsBS;
+constexpr int kSfbCols = kBN / 32;
+constexpr int kSfbCol0 = kSfaCol0 + kStages * 4;
+static_assert(kSfbCol0 + kStages * 8 <= kTmemCols, "TMEM budget (block-scaled)");
+static_assert(kSfbCols <= 8, "scale-factor columns of the token tile");
 static_assert(kBN % 32 == 0 && kBN <= 256, "token tile");
 static_assert(kWStages % 2 == 0 && kStages % 2 == 0, "ring depths must be even");
 
@@ -139,22 +148,6 @@ __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const in
   o.feat0 = o.fb * kBM;
 }
 
-// In-register transpose-reduction: on entry v[c] is this lane's term for column c; on
-// exit v[0] holds, in lane l, the sum over the 32 lanes of the terms for column l.
-__device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < off; ++i) {
-      const float send = upper ? v[i] : v[i + off];
-      const float keep = upper ? v[i + off] : v[i];
-      v[i] = keep + __shfl_xor_sync(kFull, send, off);
-    }
-  }
-  return v[0];
-}
-
 // Last-phase parity of a ring stage after `issued` uses in total (for the exit drains).
 MOE_DEV bool drain_ring(uint64_t* full, int stages, int issued, const DevErr& err, int where) {
   bool ok = true;
@@ -165,10 +158,12 @@ MOE_DEV bool drain_ring(uint64_t* full, int stages, int issued, const DevErr& er
   return ok;
 }
 
-template <int EPI, bool COLT>
+template <int EPI, bool COLT, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_tok,
+                        const __grid_constant__ CUtensorMap tmap_lo,
                         const __grid_constant__ CUtensorMap tmap_w, const GemmArgs p) {
+  static_assert(!BS || (EPI == kEpiGateUp && !COLT), "block-scaled form: gate_up only");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -177,7 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 8);
   int* s_off = reinterpret_cast<int*>(smem + SmemLayout::tables);
   int* s_tstart = s_off + 257;
-  const int sc_bytes = 4 * p.K;  // 128 rows x K/32 (per-row) or 4 x K (transposed)
+  // per tile: 128 rows x K/32 (per-row) or 4 x K (transposed) weight scales; the block-scaled
+  // form appends the token tile's activation scales (kBN rows x sfb_stride)
+  const int sc_bytes = 4 * p.K + (BS ? kBN * p.sfb_stride : 0);
   uint8_t* s_sc = smem + SmemLayout::sc;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -235,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       if (lane == 0) {
         prefetch_tmap(&tmap_tok);
+        if (BS) prefetch_tmap(&tmap_lo);
         bool ok = true;
         int s = 0;
         uint32_t ph = 0;
@@ -245,8 +243,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait_sleep(smem_u32(&bar->empty[s]), ph ^ 1, err, 0x201, s_abort, 64)) { ok = false; break; }
             const uint32_t fb = smem_u32(&bar->full[s]);
             mbar_arrive_expect_tx(fb, kTokBytes);
-            tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
-                        tl.row0, fb);
+            if (BS) {  // hi and lo E4M3 parts: 64 bytes per row each, half a stage apiece
+              tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
+                          tl.row0, fb);
+              tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes + kTokBytes / 2),
+                          &tmap_lo, ks * kBK, tl.row0, fb);
+            } else {
+              tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
+                          tl.row0, fb);
+            }
             ++issued;
             if (++s == kStages) { s = 0; ph ^= 1; }
           }
@@ -281,8 +286,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             bytes = (uint32_t)rows * kb32;
             src = p.scales + ((size_t)tl.e * N + tl.feat0) * kb32;
           }
-          mbar_arrive_expect_tx(smem_u32(&bar->sc_full[sb]), bytes);
+          const uint32_t sfb_bytes = BS ? (uint32_t)(tl.n_valid * p.sfb_stride) : 0u;
+          mbar_arrive_expect_tx(smem_u32(&bar->sc_full[sb]), bytes + sfb_bytes);
           bulk_load(smem_u32(s_sc + sb * sc_bytes), src, bytes, smem_u32(&bar->sc_full[sb]));
+          if (BS)
+            bulk_load(smem_u32(s_sc + sb * sc_bytes + 4 * K),
+                      p.sfb + (size_t)tl.row0 * p.sfb_stride, sfb_bytes,
+                      smem_u32(&bar->sc_full[sb]));
           ++sc_issued;
           for (int ks = 0; ks < nk; ++ks) {
             if (!mbar_wait_sleep(smem_u32(&bar->w_empty[ws]), wph ^ 1, err, 0x202, s_abort, 64)) { ok = false; break; }
@@ -330,7 +340,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            {
+            if (BS) {
+              // per 32-element block: the hi part, then the lo part accumulated on top, both
+              // with the stage's scale factors (byte kk of its scale columns)
+              const int npad = (tl.n_valid + 15) & ~15;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                if (h == 1 && !two) break;
+                const int st = h ? s1 : s;
+                const uint32_t tbase = tok_base + st * kTokBytes;
+                const uint64_t bhi = smem_desc_kmajor_sw64(tbase);
+                const uint64_t blo = smem_desc_kmajor_sw64(tbase + kTokBytes / 2);
+                const uint32_t a_tmem = tmem + kACol0 + st * kAColsBS;
+                const uint32_t sfa = tmem + kSfaCol0 + st * 4, sfb = tmem + kSfbCol0 + st * 8;
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                  const uint32_t id = idesc_mxf4a_m128(npad, (uint32_t)kk);
+                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, bhi + (uint64_t)(kk * 2), id, sfa, sfb,
+                              (ks | h | kk) != 0);
+                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, blo + (uint64_t)(kk * 2), id, sfa, sfb, 1u);
+                }
+                mma_commit(smem_u32(&bar->empty[st]));
+              }
+            } else {
               const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + s * kTokBytes);
               const uint32_t a_tmem = tmem + kACol0 + s * (kBK / 2);
 #pragma unroll
@@ -340,12 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_commit(smem_u32(&bar->empty[s]));
             }
             if (two) {
-              const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + s1 * kTokBytes);
-              const uint32_t a_tmem = tmem + kACol0 + s1 * (kBK / 2);
+              if (!BS) {
+                const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + s1 * kTokBytes);
+                const uint32_t a_tmem = tmem + kACol0 + s1 * (kBK / 2);
 #pragma unroll
-              for (int kk = 0; kk < kBK / 16; ++kk)
-                mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc, 1u);
-              mma_commit(smem_u32(&bar->empty[s1]));
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                  mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc, 1u);
+                mma_commit(smem_u32(&bar->empty[s1]));
+              }
               s = (s1 + 1 == kStages) ? 0 : s1 + 1;
               ph = (s1 + 1 == kStages) ? (ph1 ^ 1) : ph1;
             } else {
@@ -398,9 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // scale factors: f1 (and f2 when some scale is above 128), as bf16x2 words
         // (per row, forward: the pair's four 32-element blocks; the rare second factor is
         // re-derived from the scale bytes where it is needed)
-        uint32_t f1[4];
-        bool slow;
-        if (!COLT) {
+        uint32_t f1[4] = {0, 0, 0, 0};
+        bool slow = false;
+        if (BS) {
+          // the block-scaled MMA applies the UE8M0 scales itself (scale-factor columns)
+        } else if (!COLT) {
           uint32_t mx = 0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -454,6 +490,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((swz ^ 1) << 4));
             qw[0] = w0.x; qw[1] = w0.y; qw[2] = w0.z; qw[3] = w0.w;
             qw[4] = w1.x; qw[5] = w1.y; qw[6] = w1.z; qw[7] = w1.w;
+          }
+          if (BS) {
+            // E2M1 codes into 8-bit containers (the MMA decodes them with the scales)
+            uint32_t out16[16];
+            if (active) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) e2m1x8_to_containers(qw[i], out16[2 * i], out16[2 * i + 1]);
+            }
+            // scale factors of the k-step's two 32-element blocks, bytes 0 and 1 of a column.
+            // The MMA reads weight row m's from lane m, column m / 32: this warp's rows are
+            // its own lanes, column q.  The token tile's are read from lane n % 32, column
+            // n / 32; every lane quarter gets the same copy.
+            const int blk0 = 2 * (ks0 + h);
+            uint32_t sfa1;
+            {
+              const bool rv = r < min(kBM, N - tl.feat0);
+              const uint32_t b0 = (rv && blk0 < kb32) ? scb[r * kb32 + blk0] : 0u;
+              const uint32_t b1 = (rv && blk0 + 1 < kb32) ? scb[r * kb32 + blk0 + 1] : 0u;
+              sfa1 = b0 | (b1 << 8);
+            }
+            const uint8_t* sfbb = scb + 4 * K;
+            uint32_t sfb8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int tok = 32 * j + lane;
+              sfb8[j] = (j < kSfbCols && tok < tl.n_valid)
+                            ? *reinterpret_cast<const uint16_t*>(sfbb + tok * p.sfb_stride + blk0)
+                            : 0u;
+            }
+            const int sa = (ga + h) % kStages;
+            if (!mbar_wait(smem_u32(&bar->empty[sa]), (((ga + h) / kStages) & 1) ^ 1, err, 0x402,
+                           s_abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (active) tmem_st16(tmem + lanes + kACol0 + sa * kAColsBS, out16);
+            tmem_st1(tmem + lanes + kSfaCol0 + sa * 4 + q, sfa1);
+            tmem_st8(tmem + lanes + kSfbCol0 + sa * 8, sfb8);
+            continue;
           }
           uint32_t out[32];
           if (active) {
@@ -511,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (active) tmem_st32(tmem + lanes + kACol0 + sa * (kBK / 2), out);
         }
         if (!ok) break;
-        if (active) tmem_wait_st();
+        if (active || BS) tmem_wait_st();
         tc_fence_before();
         // packed bytes consumed and A stages written: release the weight stages and publish
         // the A stages (this also orders the pair's reads of cw before the next pair's writes)
@@ -682,10 +758,10 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int EPI, bool COLT>
-cudaError_t launch_one(const CUtensorMap& tt, const CUtensorMap& tw, const GemmArgs& a, int grid,
-                       size_t smem, cudaStream_t st) {
-  auto kern = grouped_gemm_kernel<EPI, COLT>;
+template <int EPI, bool COLT, bool BS>
+cudaError_t launch_one(const CUtensorMap& tt, const CUtensorMap& tl, const CUtensorMap& tw,
+                       const GemmArgs& a, int grid, size_t smem, cudaStream_t st) {
+  auto kern = grouped_gemm_kernel<EPI, COLT, BS>;
   // the setmaxnreg split assumes kLaunchRegs registers per thread at launch
   cudaFuncAttributes fa;
   cudaError_t fe = cudaFuncGetAttributes(&fa, kern);
@@ -694,51 +770,64 @@ cudaError_t launch_one(const CUtensorMap& tt, const CUtensorMap& tw, const GemmA
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(tt, tw, a);
+  kern<<<grid, kThreads, smem, st>>>(tt, tl, tw, a);
   return cudaGetLastError();
+}
+
+// 2-D tiled map over a row-major [rows][cols] array of `elem`-byte elements.
+bool encode_2d(EncodeTiledFn enc, CUtensorMap* m, CUtensorMapDataType type, const void* base,
+               int elem, uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+               CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
-size_t grouped_gemm_smem_bytes(int K) {
-  return 1024 + SmemLayout::sc + 2 * (size_t)(4 * K);
+size_t grouped_gemm_smem_bytes(int K, int sfb_stride) {
+  return 1024 + SmemLayout::sc + 2 * ((size_t)(4 * K) + (size_t)kBN * sfb_stride);
 }
 
-cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const uint16_t* tokens,
+cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const void* tokens,
                                 const uint8_t* wq, const GemmArgs& a, int num_sms,
                                 cudaStream_t st) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap tt, tw;
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.A};
-    const cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBN};
-    const cuuint32_t es[2] = {1, 1};
-    if (enc(&tt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(tokens), dims, strides,
-            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  const bool bs = a.tok_lo != nullptr;
+  CUtensorMap tt, tl, tw;
+  if (bs) {  // E4M3 hi / lo parts: [A][K] bytes each, 64-byte rows per k-step
+    if (epi != kEpiGateUp || transposed_scales || !a.sfb || a.sfb_stride % 16 ||
+        a.sfb_stride < 2 * ((a.K + kBK - 1) / kBK))
       return cudaErrorInvalidValue;
-  }
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
-    const cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
-    const cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), (cuuint32_t)kBM};
-    const cuuint32_t es[2] = {1, 1};
-    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(wq), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (!encode_2d(enc, &tt, CU_TENSOR_MAP_DATA_TYPE_UINT8, tokens, 1, a.K, a.A, kBK, kBN,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_2d(enc, &tl, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.tok_lo, 1, a.K, a.A, kBK, kBN,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
+  } else {
+    if (!encode_2d(enc, &tt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, tokens, 2, a.K, a.A, kBK, kBN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    tl = tt;
   }
-  const size_t smem = grouped_gemm_smem_bytes(a.K);
+  if (!encode_2d(enc, &tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, 1, a.K / 2,
+                 (uint64_t)a.E * (uint64_t)a.N, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
+  const size_t smem = grouped_gemm_smem_bytes(a.K, bs ? a.sfb_stride : 0);
   const int grid = num_sms;
+  if (bs) return launch_one<kEpiGateUp, false, true>(tt, tl, tw, a, grid, smem, st);
   switch (epi * 2 + (transposed_scales ? 1 : 0)) {
-    case kEpiGateUp * 2 + 0: return launch_one<kEpiGateUp, false>(tt, tw, a, grid, smem, st);
-    case kEpiDown * 2 + 0: return launch_one<kEpiDown, false>(tt, tw, a, grid, smem, st);
-    case kEpiDact * 2 + 1: return launch_one<kEpiDact, true>(tt, tw, a, grid, smem, st);
-    case kEpiDx * 2 + 1: return launch_one<kEpiDx, true>(tt, tw, a, grid, smem, st);
+    case kEpiGateUp * 2 + 0: return launch_one<kEpiGateUp, false, false>(tt, tl, tw, a, grid, smem, st);
+    case kEpiDown * 2 + 0: return launch_one<kEpiDown, false, false>(tt, tl, tw, a, grid, smem, st);
+    case kEpiDact * 2 + 1: return launch_one<kEpiDact, true, false>(tt, tl, tw, a, grid, smem, st);
+    case kEpiDx * 2 + 1: return launch_one<kEpiDx, true, false>(tt, tl, tw, a, grid, smem, st);
     // plain product over the stored rows (the grouped matmul entry point)
-    case kEpiDx * 2 + 0: return launch_one<kEpiDx, false>(tt, tw, a, grid, smem, st);
+    case kEpiDx * 2 + 0: return launch_one<kEpiDx, false, false>(tt, tl, tw, a, grid, smem, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -26,17 +26,24 @@ struct GemmArgs {
   uint16_t* out1;          // act [A][I] (kEpiGateUp)
   const uint32_t* dgu;     // saved GLU derivative factors [A][I] bf16x2 (kEpiDact)
   const float* w_row;      // [A] routing weight of each expert-sorted row (kEpiDact)
+  // block-scaled gate_up: the token tile comes as E4M3 hi (`tokens`) and lo parts with one
+  // UE8M0 scale per row and 32 elements (sfb [A][sfb_stride]); null for the bf16 form
+  const uint8_t* tok_lo;
+  const uint8_t* sfb;
+  int sfb_stride;
   float alpha, limit;
   float mask_limit;        // largest fp32 x whose bf16 rounding is <= limit (clamp-mask test)
   int* err;
 };
 
-// Encodes the two tensor maps and launches one persistent grouped GEMM.
-// `tokens`: bf16 [A][K] expert-sorted rows; `wq`: packed rows uint8 [E*N][K/2].
-cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const uint16_t* tokens,
+// Encodes the tensor maps and launches one persistent grouped GEMM.
+// `tokens`: bf16 [A][K] expert-sorted rows (or, with a.tok_lo set, the E4M3 hi part [A][K]
+// bytes); `wq`: packed rows uint8 [E*N][K/2].
+cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const void* tokens,
                                 const uint8_t* wq, const GemmArgs& a, int num_sms,
                                 cudaStream_t st);
-size_t grouped_gemm_smem_bytes(int K);
+// dynamic shared memory of a launch (sfb_stride: 0 for the bf16 form)
+size_t grouped_gemm_smem_bytes(int K, int sfb_stride);
 
 // Tokens are routed in blocks of a fixed size; blk_hist holds route_blocks(T) x E counts.
 int route_blocks(int T);
@@ -56,8 +63,7 @@ cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, 
 cudaError_t launch_gather_rows(const uint16_t* src, int H, int k, const int32_t* perm, int A,
                                uint16_t* dst, float* dot_w, cudaStream_t st);
 // Gather x into expert-sorted rows as two E4M3 parts with a UE8M0 scale per 32 elements
-// (hi, lo [A][H] bytes; sfb [A][sfb_stride] bytes, the scale + 6 that the block-scaled
-// gate_up GEMM applies).
+// (hi, lo [A][H] bytes; sfb [A][sfb_stride] UE8M0 bytes).
 cudaError_t launch_gather_quant(const uint16_t* x, int H, int k, const int32_t* perm, int A,
                                 uint8_t* hi, uint8_t* lo, uint8_t* sfb, int sfb_stride,
                                 cudaStream_t st);

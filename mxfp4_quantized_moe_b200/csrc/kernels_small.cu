@@ -15,17 +15,16 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---------------------------------------------------------------------------------------
 // Router: top-k over the E logits of a token (largest first, equal logits -> lower expert
-// index), softmax over the k selected, and this block's expert histogram.  One warp per
-// token: lane l holds logits l, l+32, ... (E <= 256); each of the k rounds is a lane-local
-// best followed by a five-step butterfly argmax.  A block covers kRouteTokens consecutive
-// tokens, so its assignments are the contiguous slots [b*kRouteTokens*k, ...) and its
-// histogram (written to blk_hist[b][E], no global atomics) lets the permutation kernel place
-// them without another pass over the routing.
+// index) and softmax over the k selected.  One warp per token: lane l holds logits l, l+32,
+// ... (E <= 256); each of the k rounds is a lane-local best followed by a five-step
+// butterfly argmax.  Lane j keeps selection j and adds it to the expert histogram of the
+// token's 128-token segment (blk_hist[t / 128][e], zeroed before the launch), which lets the
+// permutation kernel place every segment's slots without another pass over the routing.
 // Source: the top-k router of the eager expert loop ("Add MXFP4 training support via a
 // dequantize-on-the-fly fallback", section "What this does"); softmax over the k values.
 // ---------------------------------------------------------------------------------------
 constexpr int kRouteThreads = 256;
-constexpr int kRouteTokens = 128;  // tokens per router / permutation block
+constexpr int kRouteTokens = 128;  // tokens per histogram segment / permutation block
 
 __device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
@@ -35,74 +34,67 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(
     const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
     float* __restrict__ w, int32_t* __restrict__ blk_hist, int32_t* __restrict__ user_idx,
     float* __restrict__ user_w) {
-  __shared__ int s_hist[256];
-  for (int e = threadIdx.x; e < E; e += kRouteThreads) s_hist[e] = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t_end = min(T, (blockIdx.x + 1) * kRouteTokens);
-  for (int t = blockIdx.x * kRouteTokens + warp; t < t_end; t += kRouteThreads / 32) {
-    const float* row = logits + (size_t)t * E;
-    float v[8];
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * kRouteThreads + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const float* row = logits + (size_t)t * E;
+  float v[8];
+  uint32_t taken = 0;  // bit i: expert lane + 32 i already selected (or absent)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      const float x = (e < E) ? __ldg(row + e) : -INFINITY;
-      v[i] = (x != x) ? -INFINITY : x;  // a NaN logit is never preferred
-    }
-    uint32_t taken = 0;  // bit i: expert lane + 32 i already selected (or absent)
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    const float x = (e < E) ? __ldg(row + e) : -INFINITY;
+    v[i] = (x != x) ? -INFINITY : x;  // a NaN logit is never preferred
+    if (e >= E) taken |= 1u << i;
+  }
+  float m0 = 0.f, zsum = 0.f;
+  float myz = 0.f;  // selection `lane` (k <= 32); lane j % 32 parks selections j >= 32 in
+  int myi = 0;      // idx / w until the softmax denominator is known
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7FFFFFFF;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      if (lane + 32 * i >= E) taken |= 1u << i;
-    float m0 = 0.f, zsum = 0.f;
-    float zr[8];
-    int ir[8];
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7FFFFFFF;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (!(taken & (1u << i)) && beats(v[i], lane + 32 * i, bv, bi)) {
-          bv = v[i];
-          bi = lane + 32 * i;
-        }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(kFull, bv, o);
-        const int oi = __shfl_xor_sync(kFull, bi, o);
-        if (beats(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
+      if (!(taken & (1u << i)) && beats(v[i], lane + 32 * i, bv, bi)) {
+        bv = v[i];
+        bi = lane + 32 * i;
       }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (j == 0) m0 = bv;
-      const float z = __expf(bv - m0);
-      zsum += z;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (i == (j >> 5) && lane == (j & 31)) {
-          zr[i] = z;
-          ir[i] = bi;
-        }
-      if (lane == 0) atomicAdd(&s_hist[bi], 1);
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(kFull, bv, o);
+      const int oi = __shfl_xor_sync(kFull, bi, o);
+      if (beats(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
     }
-    const float inv = 1.f / zsum;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int j = 32 * i + lane;
-      if (j < k) {
-        const size_t o = (size_t)t * k + j;
-        const float wj = zr[i] * inv;
-        idx[o] = ir[i];
-        w[o] = wj;
-        if (user_idx) user_idx[o] = ir[i];
-        if (user_w) user_w[o] = wj;
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (j == 0) m0 = bv;
+    const float z = __expf(bv - m0);
+    zsum += z;
+    if (lane == (j & 31)) {
+      if (j < 32) {
+        myz = z;
+        myi = bi;
+      } else {
+        w[(size_t)t * k + j] = z;
+        idx[(size_t)t * k + j] = bi;
       }
     }
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kRouteThreads)
-    blk_hist[(size_t)blockIdx.x * E + e] = s_hist[e];
+  const float inv = 1.f / zsum;
+  int32_t* hist = blk_hist + (size_t)(t / kRouteTokens) * E;
+  for (int j = lane; j < k; j += 32) {
+    const size_t o = (size_t)t * k + j;
+    const float z = (j < 32) ? myz : w[o];
+    const int e = (j < 32) ? myi : idx[o];
+    const float wj = z * inv;
+    idx[o] = e;
+    w[o] = wj;
+    if (user_idx) user_idx[o] = e;
+    if (user_w) user_w[o] = wj;
+    atomicAdd(hist + e, 1);
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -124,14 +116,31 @@ __global__ void __launch_bounds__(kRouteThreads) build_perm_kernel(
   __shared__ int s_scan[kWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
-  // (a) + (b): thread e sums column e of the [nblk][E] histograms
-  int before = 0, total = 0;
+  // (a) + (b): column sums of the [nblk][E] segment histograms; `parts` threads share each
+  // expert's column (strided over the segments), then their partial sums are added
+  __shared__ int s_part[2][kRouteThreads];
   const int e = threadIdx.x;
+  {
+    const int parts = kRouteThreads / E;  // >= 1 (E <= 256)
+    const int ex = threadIdx.x % E, part = threadIdx.x / E;
+    int bf = 0, tot = 0;
+    if (part < parts) {
+#pragma unroll 4
+      for (int bb = part; bb < nblk; bb += parts) {
+        const int c = __ldg(blk_hist + (size_t)bb * E + ex);
+        tot += c;
+        bf += (bb < b) ? c : 0;
+      }
+    }
+    s_part[0][threadIdx.x] = bf;
+    s_part[1][threadIdx.x] = tot;
+    __syncthreads();
+  }
+  int before = 0, total = 0;
   if (e < E) {
-    for (int bb = 0; bb < nblk; ++bb) {
-      const int c = __ldg(blk_hist + (size_t)bb * E + e);
-      total += c;
-      if (bb < b) before += c;
+    for (int i = e; i < kRouteThreads - (kRouteThreads % E); i += E) {
+      before += s_part[0][i];
+      total += s_part[1][i];
     }
   }
   // exclusive scan of the totals over experts (E <= 256 = one value per thread)
@@ -240,8 +249,7 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ src, int H, int 
 // For every expert-sorted row r (token t = perm[r] / k) and 32-element block b of x[t]:
 //   S  = the smallest integer with max|x_block| <= 448 * 2^S (clamped to [-126, 121]),
 //   hi = e4m3(x / 2^S), lo = e4m3(x / 2^S - hi)   (round to nearest even, exact residual),
-//   sfb[r][b] = S + 133: the UE8M0 scale the MMA applies to both parts, 2^(S + 6), where the
-//   extra 2^6 undoes the weights' E2M1 -> E4M3 re-encoding (value * 2^-6) in the GEMM.
+//   sfb[r][b] = S + 127: the UE8M0 scale 2^S the MMA applies to both parts.
 // x / 2^S has at most 8 significant bits; hi keeps the top 4 and lo the next 4 (the remainder
 // is exact in fp32), so hi + lo equals x / 2^S for every element within 2^9 of the block
 // maximum that stays above the E4M3 subnormal floor; smaller elements keep an absolute error
@@ -299,7 +307,7 @@ __global__ void gather_quant_kernel(const uint16_t* __restrict__ x, int H, int k
     } else {
       const int E = (int)(amax >> 7), m7 = (int)(amax & 0x7F);
       const int S = (E == 0) ? -126 : max(-126, E - 135 + (m7 > 0x60 ? 1 : 0));
-      sbyte = S + 133;
+      sbyte = S + 127;
       const float inv = __uint_as_float((uint32_t)(127 - S) << 23);  // 2^-S, exact
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -438,8 +446,11 @@ int route_blocks(int T) { return (T + kRouteTokens - 1) / kRouteTokens; }
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
                                int32_t* blk_hist, int32_t* user_idx, float* user_w,
                                cudaStream_t st) {
-  router_topk_kernel<<<route_blocks(T), kRouteThreads, 0, st>>>(logits, T, E, k, idx, w, blk_hist,
-                                                                user_idx, user_w);
+  cudaError_t e = cudaMemsetAsync(blk_hist, 0, sizeof(int32_t) * (size_t)route_blocks(T) * E, st);
+  if (e != cudaSuccess) return e;
+  const int warps_per_block = kRouteThreads / 32;
+  router_topk_kernel<<<(T + warps_per_block - 1) / warps_per_block, kRouteThreads, 0, st>>>(
+      logits, T, E, k, idx, w, blk_hist, user_idx, user_w);
   return cudaGetLastError();
 }
 

@@ -12,7 +12,8 @@ from oracle import mxfp4_oracle as O
 def block(job):
     """One block of a stack checked on recorded inputs: job = (workload, seed, layer, x,
     logits, g) with x, logits, g the sampled tokens' block input, router logits and upstream
-    gradient as the GPU saw them.  Returns the oracle's (out, dX, d_w, d_logits, w)."""
+    gradient as the GPU saw them.  Returns the oracle's (out, dX, d_w, d_logits, w) and
+    sum_h |g_h| |y_{j,h}| per token and slot."""
     os.environ.setdefault("OMP_NUM_THREADS", "2")
     wl, seed, l, x, logits, g = job
     inp = inputs.make_workload(wl, seed, layer=l, with_dy=False)
@@ -20,4 +21,6 @@ def block(job):
     del inp
     f = O.moe_forward(x, logits, W, wl.k)
     dX, d_w, d_logits = O.moe_backward(g, f, W)
-    return np.asarray(f["out"]), dX, d_w, d_logits, f["w"]
+    # sum_h |g_h y_{j,h}| per (token, slot): the scale of the rounding of y in d_w = <g, y_j>
+    y_abs = np.einsum("th,tjh->tj", np.abs(g), np.abs(f["y"]))
+    return np.asarray(f["out"]), dX, d_w, d_logits, f["w"], y_abs

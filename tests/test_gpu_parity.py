@@ -44,17 +44,27 @@ def assert_close(got, ref, name, out_dtype=None):
     assert cos >= COS_TOL, f"{name}: cosine {cos:.7f}"
 
 
-def assert_d_logits_close(got, ref, w, d_w, name="d_logits", require_resolved=False):
+def assert_d_logits_close(got, ref, w, d_w, name="d_logits", require_resolved=False, y_abs=None):
     """d_logits[t, idx_j] = w_j (d_w_j - sum_i w_i d_w_i) cancels when routing is nearly
     one-hot: the fp32 router backward cannot resolve it below about 2^-23 max|w * d_w| per
     token, while the fp64 oracle does.  So the reference (rounded to fp32, the output's
     precision) is compared with an absolute floor of 2^-20 max|w * d_w| per token (8x the
-    fp32 resolution of the k-term sum); above the floor this is the usual per-tensor bar."""
+    fp32 resolution of the k-term sum); above the floor this is the usual per-tensor bar.
+
+    With `y_abs` (sum_h |dY_h| |y_{j,h}| per token and slot) the floor also covers the bf16
+    rounding of the expert outputs y that d_w = <dY, y_j> is taken on: each d_w_j is then off
+    by up to 2^-9 y_abs_j (plus the fp32 sum), and the Jacobian can pass twice that on, so the
+    floor is 2^-7 max_j w_j max_i y_abs_i per token."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64).astype(np.float32).astype(np.float64)
     floor = 2.0 ** -20 * np.max(np.abs(np.asarray(w, np.float64) * np.asarray(d_w, np.float64)),
                                 axis=1, keepdims=True)
-    resolved = np.abs(ref).max(axis=1, keepdims=True) > floor
+    margin = 1.0
+    if y_abs is not None:
+        wmax = np.max(np.asarray(w, np.float64), axis=1, keepdims=True)
+        floor = np.maximum(floor, 2.0 ** -7 * wmax * np.max(y_abs, axis=1, keepdims=True))
+        margin = 64.0  # the per-tensor bar only for tokens resolved well above their floor
+    resolved = np.abs(ref).max(axis=1, keepdims=True) > margin * floor
     if require_resolved:
         assert resolved.all(), f"{name}: a token's reference lies below the fp32 floor"
     # tokens whose d_logits lies below the fp32 floor: absolute bound only
@@ -306,18 +316,69 @@ def test_interleave_helper_restores_the_shipped_row_order(moe):
     assert torch.equal(obias.cpu(), inp["gu_bias"])
 
 
-def _ws_offsets(T, E, k):
-    """Offsets of the routing regions in the forward's workspace (the library's layout: each
-    region starts 256-byte aligned, in the order error word, offsets, idx, w, perm, inv)."""
+def _sfb_stride(H):
+    """Row stride of the activation scales: one byte per 32 elements, padded to whole 64-element
+    k-steps and to 16 bytes."""
+    return (2 * (-(-H // 64)) + 15) // 16 * 16
+
+
+def _ws_offsets(T, E, k, H=None, I=None):
+    """Offsets of the regions of the forward's workspace (the library's layout: each region
+    starts 256-byte aligned, in the order error word, offsets, idx, w, perm, inv, w_row, router
+    block histograms, activation scales, GLU factors, act, dH, rows)."""
     def up(v):
         return (v + 255) // 256 * 256
     A = T * k
+    sizes = [("err", 16), ("off", 4 * (E + 1)), ("idx", 4 * A), ("w", 4 * A), ("perm", 4 * A),
+             ("inv", 4 * A), ("w_row", 4 * A), ("blk_hist", 4 * (-(-T // 128)) * E)]
+    if H is not None:
+        sizes += [("sfb", A * _sfb_stride(H)), ("dgu", 4 * A * I), ("act", 2 * A * I),
+                  ("dh", 4 * A * I), ("rows", 2 * A * H)]
     o, out = 0, {}
-    for name, size in (("err", 16), ("off", 4 * (E + 1)), ("idx", 4 * A),
-                       ("w", 4 * A), ("perm", 4 * A), ("inv", 4 * A)):
+    for name, size in sizes:
         out[name] = o
         o = up(o + size)
     return out
+
+
+def _e4m3_values(b):
+    """E4M3 bytes -> values (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+    exponent field 0 is subnormal with spacing 2^-9)."""
+    b = np.asarray(b, np.int64)
+    e, m = (b >> 3) & 15, b & 7
+    mag = np.where(e > 0, np.ldexp(1.0 + m / 8.0, e - 7), np.ldexp(m / 8.0, -6))
+    return np.where(b & 0x80, -mag, mag)
+
+
+def test_activation_split_matches_the_mx_definition(moe):
+    """The gather feeding the block-scaled gate_up GEMM: each expert-sorted row of x, split per
+    32 elements into hi + lo E4M3 parts with a UE8M0 scale 2^S, bit for bit the oracle's
+    mx_split of the same row (S stored as the UE8M0 byte S + 127)."""
+    T, H, I, E, k = 300, 352, 96, 7, 3
+    inp = inputs.make_layer(T, H, I, E, k, 41)
+    x = inp["x"].clone()
+    x[5, :32] = 0.0         # an all-zero block
+    x[7, 32:64] *= 2 ** 40  # a large block
+    x[9, 64:96] *= 2 ** -40  # a small block, elements far below the rest of the row
+    shape = moe.MoeShape(T, H, I, E, k)
+    w = moe.weights_to(inp, "cuda")
+    ws = moe.alloc_workspace(shape)
+    moe.forward(shape, w, x.cuda(), inp["logits"].cuda(), ws)
+    assert moe.device_check(ws) == (0, 0)
+    o, A = _ws_offsets(T, E, k, H, I), T * k
+    wsn = ws.cpu().numpy()
+    perm = wsn[o["perm"]:o["perm"] + 4 * A].view(np.int32)
+    hi = wsn[o["rows"]:o["rows"] + A * H].reshape(A, H)
+    lo = wsn[o["rows"] + A * H:o["rows"] + 2 * A * H].reshape(A, H)
+    st = _sfb_stride(H)
+    sfb = wsn[o["sfb"]:o["sfb"] + A * st].reshape(A, st)
+    xs = O.bf16_bits_to_f64(x.view(torch.int16).numpy().view(np.uint16))[perm // k]
+    rhi, rlo, S = O.mx_split(xs)
+    S = S.reshape(A, H // 32)
+    zero = np.abs(xs).reshape(A, H // 32, 32).max(axis=2) == 0
+    assert np.array_equal(_e4m3_values(hi), rhi) and np.array_equal(_e4m3_values(lo), rlo)
+    assert np.array_equal(sfb[:, :H // 32][~zero].astype(np.int64) - 127, S[~zero])
+    assert np.all(sfb[:, H // 32:] == 0)
 
 
 def test_permutation_is_the_stable_expert_sort(moe):

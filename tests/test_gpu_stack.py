@@ -69,11 +69,20 @@ def _run_blockwise(wl, seed, sel, workers=1):
             refs = list(ex.map(oracle_pool.block, jobs))
     else:
         refs = [oracle_pool.block(j) for j in jobs]
-    for l, (out, dX, d_w, d_logits, w) in enumerate(refs):
+    for l, (out, dX, d_w, d_logits, w, y_abs) in enumerate(refs):
         assert_close(_np(fw[l]["y"]), out, f"y[{l}]")
         assert_close(_np(bw[l]["dx"]), dX, f"dx[{l}]")
-        assert_close(_np(bw[l]["d_w"]), d_w, f"d_w[{l}]", np.float32)
-        assert_d_logits_close(_np(bw[l]["d_logits"]), d_logits, w, d_w, f"d_logits[{l}]")
+        gdw = _np(bw[l]["d_w"])
+        assert_close(gdw, d_w, f"d_w[{l}]", np.float32)
+        gdl = _np(bw[l]["d_logits"])
+        # d_logits against the oracle, with the per-token floor of the bf16 rounding of y
+        assert_d_logits_close(gdl, d_logits, w, d_w, f"d_logits[{l}]", y_abs=y_abs)
+        # the softmax Jacobian itself, applied in fp64 to the GPU's own d_w: fp32-exact
+        idx = np.argsort(-fw[l]["logits"].double().numpy(), axis=1, kind="stable")[:, :wl.k]
+        sel = w * (gdw - (w * gdw).sum(axis=1, keepdims=True))
+        jac = np.zeros_like(gdl)
+        np.put_along_axis(jac, idx, sel, axis=1)
+        assert_d_logits_close(gdl, jac, w, gdw, f"d_logits[{l}] from the GPU's d_w")
 
 
 def test_small_stack_blockwise_all_tokens():
