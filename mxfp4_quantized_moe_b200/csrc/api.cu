@@ -42,9 +42,9 @@ WsLayout ws_layout(const mxfp4_moe_dims& d) {
   L.sfb = o;      o = up(o + A * sfb_stride(d.H));     // activation scales (gate_up)
   L.dgu = o;      o = up(o + 4 * A * d.I);           // saved GLU derivative factors (bf16 pairs)
   L.act = o;      o = up(o + 2 * A * d.I);           // act [A][I] (the down GEMM's input)
-  L.dh = o;       o = up(o + 2 * A * 2 * d.I);       // dH [A][2I] (backward scratch)
-  L.rows = o;     o = up(o + 2 * A * d.H);           // E4M3 hi|lo of Xp -> y (fwd),
-                                                     // dYp -> dX rows (bwd)
+  // dH [A][2I] (backward); in the forward, the E4M3 hi | lo parts of Xp ([A][H] bytes each)
+  L.dh = o;       o = up(o + 2 * A * (2 * d.I > d.H ? 2 * d.I : d.H));
+  L.rows = o;     o = up(o + 2 * A * d.H);           // y (fwd), dYp -> dX rows (bwd)
   L.total = o;
   return L;
 }
@@ -256,8 +256,9 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
 
   MOE_LAUNCH("router_topk", moe::launch_router_topk(logits, T, E, k, idx, wr, blk_hist, topk_idx, topk_w, st));
   MOE_LAUNCH("build_perm", moe::launch_build_perm(idx, wr, T, E, k, blk_hist, off, perm, inv, w_row, err, st));
-  // Xp in expert-sorted order as two E4M3 parts (hi | lo in `rows`) with UE8M0 block scales
-  uint8_t* xhi = reinterpret_cast<uint8_t*>(rows);
+  // Xp in expert-sorted order as two E4M3 parts (hi | lo in the dH region, free until the
+  // backward) with UE8M0 block scales
+  uint8_t* xhi = at<uint8_t>(ws, L.dh);
   uint8_t* xlo = xhi + (size_t)A * H;
   uint8_t* sfb = at<uint8_t>(ws, L.sfb);
   MOE_LAUNCH("gather_x_mx", moe::launch_gather_quant(x, H, k, perm, A, xhi, xlo, sfb, sfb_stride(H), st));

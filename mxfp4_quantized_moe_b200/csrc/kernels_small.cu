@@ -215,6 +215,14 @@ __global__ void __launch_bounds__(kRouteThreads) build_perm_kernel(
 // reads a 16-byte chunk of y_r and then writes the same chunk, and no other lane or warp
 // touches that chunk, so reading and writing one buffer is safe.
 // ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf16x8_dot(const uint4& a, const uint4& b) {
+  float acc = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x);
+  acc += bf16_lo(a.y) * bf16_lo(b.y) + bf16_hi(a.y) * bf16_hi(b.y);
+  acc += bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z);
+  acc += bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
+  return acc;
+}
+
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ src, int H, int k,
                                    const int32_t* __restrict__ perm, int A, uint16_t* dst,
                                    float* __restrict__ dot_w) {
@@ -227,16 +235,27 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ src, int H, int 
   uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * H);
   const int nv = H / 8;
   float acc = 0.f;
-  for (int i = lane; i < nv; i += 32) {
-    const uint4 v = __ldg(s + i);
-    if (dot_w) {
-      const uint4 y = d[i];
-      acc += bf16_lo(v.x) * bf16_lo(y.x) + bf16_hi(v.x) * bf16_hi(y.x);
-      acc += bf16_lo(v.y) * bf16_lo(y.y) + bf16_hi(v.y) * bf16_hi(y.y);
-      acc += bf16_lo(v.z) * bf16_lo(y.z) + bf16_hi(v.z) * bf16_hi(y.z);
-      acc += bf16_lo(v.w) * bf16_lo(y.w) + bf16_hi(v.w) * bf16_hi(y.w);
+  // four 16-byte chunks per lane in flight: all loads of a group are issued before its stores
+  // (the chunks are distinct, so reading y and writing dY in place keeps its order per chunk)
+  constexpr int kG = 4;
+  for (int i0 = lane; i0 < nv; i0 += 32 * kG) {
+    uint4 v[kG], y[kG];
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      const int i = i0 + 32 * g;
+      if (i < nv) {
+        v[g] = __ldg(s + i);
+        if (dot_w) y[g] = d[i];
+      }
     }
-    d[i] = v;
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      const int i = i0 + 32 * g;
+      if (i < nv) {
+        if (dot_w) acc += bf16x8_dot(v[g], y[g]);
+        d[i] = v[g];
+      }
+    }
   }
   if (dot_w) {
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
@@ -361,21 +380,27 @@ __global__ void combine_kernel(const uint16_t* __restrict__ rows, const int32_t*
 }
 
 // d_logits through the softmax over the k selected logits:
-// d_l[idx_j] = w_j (d_w_j - sum_i w_i d_w_i), 0 for the experts not selected.
+// d_l[idx_j] = w_j (d_w_j - sum_i w_i d_w_i), 0 for the experts not selected.  One thread per
+// output element (token t, expert e), so that the [T][E] stores are coalesced; the k-term
+// sums are re-read from L1 by the E threads of a token.
 __global__ void router_backward_kernel(const int32_t* __restrict__ idx,
                                        const float* __restrict__ w,
                                        const float* __restrict__ d_topk_w, int T, int E, int k,
                                        float* __restrict__ d_logits) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  float s = 0.f;
-  for (int j = 0; j < k; ++j) s += w[t * k + j] * d_topk_w[t * k + j];
-  float* dl = d_logits + (size_t)t * E;
-  for (int e = 0; e < E; ++e) dl[e] = 0.f;
+  const size_t n = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= (size_t)T * E) return;
+  const int t = (int)(n / E), e = (int)(n % E);
+  const int32_t* it = idx + (size_t)t * k;
+  const float* wt = w + (size_t)t * k;
+  const float* dt = d_topk_w + (size_t)t * k;
+  float s = 0.f, out = 0.f;
+  int mine = -1;
   for (int j = 0; j < k; ++j) {
-    const int slot = t * k + j;
-    dl[idx[slot]] = w[slot] * (d_topk_w[slot] - s);
+    s += __ldg(wt + j) * __ldg(dt + j);
+    if (__ldg(it + j) == e) mine = j;
   }
+  if (mine >= 0) out = __ldg(wt + mine) * (__ldg(dt + mine) - s);
+  d_logits[n] = out;
 }
 
 // One thread per 8 elements (one 32-bit word of codes, a quarter of an MX block): a warp reads
@@ -491,7 +516,9 @@ cudaError_t launch_combine(const uint16_t* rows, const int32_t* inv, const float
 cudaError_t launch_router_backward(const int32_t* idx, const float* w, const float* d_topk_w,
                                    int T, int E, int k, float* d_logits, cudaStream_t st) {
   if (!d_logits) return cudaSuccess;
-  router_backward_kernel<<<(T + 127) / 128, 128, 0, st>>>(idx, w, d_topk_w, T, E, k, d_logits);
+  const size_t n = (size_t)T * E;
+  router_backward_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(idx, w, d_topk_w, T, E, k,
+                                                                     d_logits);
   return cudaGetLastError();
 }
 

@@ -333,7 +333,7 @@ def _ws_offsets(T, E, k, H=None, I=None):
              ("inv", 4 * A), ("w_row", 4 * A), ("blk_hist", 4 * (-(-T // 128)) * E)]
     if H is not None:
         sizes += [("sfb", A * _sfb_stride(H)), ("dgu", 4 * A * I), ("act", 2 * A * I),
-                  ("dh", 4 * A * I), ("rows", 2 * A * H)]
+                  ("dh", 2 * A * max(2 * I, H)), ("rows", 2 * A * H)]
     o, out = 0, {}
     for name, size in sizes:
         out[name] = o
@@ -368,8 +368,8 @@ def test_activation_split_matches_the_mx_definition(moe):
     o, A = _ws_offsets(T, E, k, H, I), T * k
     wsn = ws.cpu().numpy()
     perm = wsn[o["perm"]:o["perm"] + 4 * A].view(np.int32)
-    hi = wsn[o["rows"]:o["rows"] + A * H].reshape(A, H)
-    lo = wsn[o["rows"] + A * H:o["rows"] + 2 * A * H].reshape(A, H)
+    hi = wsn[o["dh"]:o["dh"] + A * H].reshape(A, H)  # the forward leaves them in the dH region
+    lo = wsn[o["dh"] + A * H:o["dh"] + 2 * A * H].reshape(A, H)
     st = _sfb_stride(H)
     sfb = wsn[o["sfb"]:o["sfb"] + A * st].reshape(A, st)
     xs = O.bf16_bits_to_f64(x.view(torch.int16).numpy().view(np.uint16))[perm // k]
