@@ -25,12 +25,6 @@
 // TMEM (512 columns): two fp32 accumulators of kBN columns (double buffered across tiles)
 // and a 4-stage ring of A operands (32 columns = 64 bf16 of K each).
 //
-// Paired form (PAIR): a tile takes up to 2 x kBN token rows as two sub-tiles that share every
-// converted A stage, so each expansion of the weights feeds twice the MMA work.  The two
-// accumulators then hold the two sub-tiles of one tile (no double buffering across tiles:
-// the next tile's MMAs wait for the epilogue), and the token ring is decoupled from the A
-// ring and counts sub-tiles (kTokStagesP stages of one sub-tile each).
-//
 // Which weights: the forward GEMMs read the stored rows (scales per row and 32-element
 // block of K).  The backward GEMMs contract over the stored rows' output axis, so they
 // read the transposed copy (element (n, k) of W^T); there the 32-element scale blocks run
@@ -55,8 +49,6 @@ namespace {
 // (TMEM) of one k-step; the MMA waits once and commits once per k-step.
 constexpr int kStages = 4;        // even: a stage always belongs to the same converter parity
 constexpr int kWStages = 8;       // packed-weight ring depth (even, same reason)
-constexpr int kTokStagesP = 6;    // paired form: token ring of sub-tile stages
-constexpr int kWStagesP = 6;      // paired form: packed-weight ring depth (even)
 constexpr int kThreads = 512;
 constexpr int kConvWarps = 8;
 constexpr int kTokBytes = kBN * kBK * 2;      // 24 KB
@@ -93,12 +85,9 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 
 struct __align__(8) Barriers {
   uint64_t full[kStages];   // token bytes landed + 4 converter warps stored the A operand
-                            // (paired form: the 4 converter warps only)
   uint64_t empty[kStages];  // MMA commit: token stage and A stage free again
   uint64_t w_full[kWStages];
   uint64_t w_empty[kWStages];
-  uint64_t tok_full[kTokStagesP];   // paired form: sub-tile bytes landed
-  uint64_t tok_empty[kTokStagesP];  // paired form: MMA commit of the sub-tile's k-step
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t sc_full[2];
@@ -107,21 +96,17 @@ struct __align__(8) Barriers {
 };
 static_assert(sizeof(Barriers) <= 512, "barrier block");
 
-template <bool PAIR>
-struct SmemLayoutT {
-  static constexpr int tok_stages = PAIR ? kTokStagesP : kStages;
-  static constexpr int w_stages = PAIR ? kWStagesP : kWStages;
+struct SmemLayout {
   // offsets from the 1024-aligned dynamic smem base
   static constexpr int tok = 0;                                  // 1024-aligned (128B swizzle)
-  static constexpr int w = tok + tok_stages * kTokBytes;         // 256-aligned (32B swizzle)
-  static constexpr int bars = w + w_stages * kWBytes;
+  static constexpr int w = tok + kStages * kTokBytes;            // 256-aligned (32B swizzle)
+  static constexpr int bars = w + kWStages * kWBytes;
   static constexpr int misc = bars + 512;                        // tmem slot, abort flag
   static constexpr int cw = misc + 64;                           // 8 warps x 4 x 32 scale words
   static constexpr int tables = cw + kConvWarps * 4 * 32 * 4;    // off[257], tile_start[257]
   static constexpr int sc = ((tables + 2 * 257 * 4) + 127) / 128 * 128;  // 2 scale buffers
 };
-static_assert(SmemLayoutT<false>::w % 1024 == 0 && SmemLayoutT<true>::w % 1024 == 0,
-              "weight ring alignment");
+static_assert(SmemLayout::w % 1024 == 0, "weight ring alignment");
 
 template <uint32_t N>
 MOE_DEV void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
@@ -130,27 +115,23 @@ MOE_DEV void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0
 
 struct Tile {
   int e, fb, row0, n_valid, feat0;
-  int n0, n1;  // sub-tile rows (paired form; otherwise n0 = n_valid, n1 = 0)
 };
 
-// An expert's m rows are split into equal token tiles of at most `cap` rows (kBN, or 2 kBN
-// in the paired form), a multiple of 16, so that no tile is a small remainder: the MMA costs
-// nearly the same at N = 64 as at N = 192.
-MOE_DEV int token_tile_rows(int m, int cap) {
-  const int n = (m + cap - 1) / cap;
+// An expert's m rows are split into equal token tiles of at most kBN rows (a multiple of 16),
+// so that no tile is a small remainder: the MMA costs nearly the same at N = 64 as at N = 192.
+MOE_DEV int token_tile_rows(int m) {
+  const int n = (m + kBN - 1) / kBN;
   const int rows = (m + n - 1) / n;
   return (rows + 15) & ~15;
 }
-MOE_DEV int token_tiles(int m, int cap) {
+MOE_DEV int token_tiles(int m) {
   if (m <= 0) return 0;
-  const int rows = token_tile_rows(m, cap);
+  const int rows = token_tile_rows(m);
   return (m + rows - 1) / rows;
 }
 
-template <bool PAIR>
 __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const int* s_off, int E,
                                             int nfb, Tile& o) {
-  constexpr int cap = PAIR ? 2 * kBN : kBN;
   int lo = 0, hi = E;  // largest lo with s_tstart[lo] <= t (s_tstart[E] = total > t)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -159,19 +140,12 @@ __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const in
   const int local = t - s_tstart[lo];
   const int tt = local / nfb;
   const int m = s_off[lo + 1] - s_off[lo];
-  const int rows = token_tile_rows(m, cap);
+  const int rows = token_tile_rows(m);
   o.e = lo;
   o.fb = local - tt * nfb;
   o.row0 = s_off[lo] + tt * rows;
   o.n_valid = min(rows, m - tt * rows);
   o.feat0 = o.fb * kBM;
-  if (PAIR && o.n_valid > kBN) {
-    o.n0 = ((o.n_valid + 1) / 2 + 15) & ~15;  // <= kBN since n_valid <= 2 kBN
-    o.n1 = o.n_valid - o.n0;
-  } else {
-    o.n0 = o.n_valid;
-    o.n1 = 0;
-  }
 }
 
 // Last-phase parity of a ring stage after `issued` uses in total (for the exit drains).
@@ -184,27 +158,24 @@ MOE_DEV bool drain_ring(uint64_t* full, int stages, int issued, const DevErr& er
   return ok;
 }
 
-template <int EPI, bool COLT, bool BS, bool PAIR>
+template <int EPI, bool COLT, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_tok,
                         const __grid_constant__ CUtensorMap tmap_lo,
                         const __grid_constant__ CUtensorMap tmap_w, const GemmArgs p) {
   static_assert(!BS || (EPI == kEpiGateUp && !COLT), "block-scaled form: gate_up only");
-  static_assert(!(BS && PAIR), "the paired form takes bf16 token tiles");
-  using SL = SmemLayoutT<PAIR>;
-  constexpr int WST = SL::w_stages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  Barriers* bar = reinterpret_cast<Barriers*>(smem + SL::bars);
-  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + SL::misc);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SL::misc + 8);
-  int* s_off = reinterpret_cast<int*>(smem + SL::tables);
+  Barriers* bar = reinterpret_cast<Barriers*>(smem + SmemLayout::bars);
+  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + SmemLayout::misc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 8);
+  int* s_off = reinterpret_cast<int*>(smem + SmemLayout::tables);
   int* s_tstart = s_off + 257;
   // per tile: 128 rows x K/32 (per-row) or 4 x K (transposed) weight scales; the block-scaled
   // form appends the token tile's activation scales (kBN rows x sfb_stride)
   const int sc_bytes = 4 * p.K + (BS ? kBN * p.sfb_stride : 0);
-  uint8_t* s_sc = smem + SL::sc;
+  uint8_t* s_sc = smem + SmemLayout::sc;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const DevErr err{p.err};
@@ -219,16 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *s_abort = 0;
     mbar_init(smem_u32(&bar->drain), 1);
     for (int s = 0; s < kStages; ++s) {
-      // token producer (not in the paired form) + 4 converter warps
-      mbar_init(smem_u32(&bar->full[s]), PAIR ? 4 : 1 + 4);
+      mbar_init(smem_u32(&bar->full[s]), 1 + 4);  // token producer + 4 converter warps
       mbar_init(smem_u32(&bar->empty[s]), 1);     // MMA commit
     }
-    if (PAIR)
-      for (int s = 0; s < kTokStagesP; ++s) {
-        mbar_init(smem_u32(&bar->tok_full[s]), 1);
-        mbar_init(smem_u32(&bar->tok_empty[s]), 1);
-      }
-    for (int s = 0; s < WST; ++s) {
+    for (int s = 0; s < kWStages; ++s) {
       mbar_init(smem_u32(&bar->w_full[s]), 1);
       mbar_init(smem_u32(&bar->w_empty[s]), 4);  // the 4 converter warps of this parity
     }
@@ -249,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       s_tstart[e] = acc;
-      acc += token_tiles(s_off[e + 1] - s_off[e], PAIR ? 2 * kBN : kBN) * nfb;
+      acc += token_tiles(s_off[e + 1] - s_off[e]) * nfb;
     }
     s_tstart[E] = acc;
   }
@@ -273,33 +238,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ph = 0;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
           Tile tl;
-          decode_tile<PAIR>(t, s_tstart, s_off, E, nfb, tl);
-          if (PAIR) {
-            // one stage per sub-tile and k-step, in the order the MMA issuer consumes them
-            for (int ks = 0; ks < nk && ok; ++ks) {
-              for (int j = 0; j < 2; ++j) {
-                if (j == 1 && tl.n1 == 0) break;
-                if (!mbar_wait_sleep(smem_u32(&bar->tok_empty[s]), ph ^ 1, err, 0x203, s_abort, 64)) { ok = false; break; }
-                const uint32_t fb = smem_u32(&bar->tok_full[s]);
-                mbar_arrive_expect_tx(fb, kTokBytes);
-                tma_load_2d(smem_u32(smem + SL::tok + s * kTokBytes), &tmap_tok, ks * kBK,
-                            tl.row0 + (j ? tl.n0 : 0), fb);
-                ++issued;
-                if (++s == kTokStagesP) { s = 0; ph ^= 1; }
-              }
-            }
-          }
-          for (int ks = 0; ks < nk && !PAIR; ++ks) {
+          decode_tile(t, s_tstart, s_off, E, nfb, tl);
+          for (int ks = 0; ks < nk; ++ks) {
             if (!mbar_wait_sleep(smem_u32(&bar->empty[s]), ph ^ 1, err, 0x201, s_abort, 64)) { ok = false; break; }
             const uint32_t fb = smem_u32(&bar->full[s]);
             mbar_arrive_expect_tx(fb, kTokBytes);
             if (BS) {  // hi and lo E4M3 parts: 64 bytes per row each, half a stage apiece
-              tma_load_2d(smem_u32(smem + SL::tok + s * kTokBytes), &tmap_tok, ks * kBK,
+              tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
                           tl.row0, fb);
-              tma_load_2d(smem_u32(smem + SL::tok + s * kTokBytes + kTokBytes / 2),
+              tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes + kTokBytes / 2),
                           &tmap_lo, ks * kBK, tl.row0, fb);
             } else {
-              tma_load_2d(smem_u32(smem + SL::tok + s * kTokBytes), &tmap_tok, ks * kBK,
+              tma_load_2d(smem_u32(smem + SmemLayout::tok + s * kTokBytes), &tmap_tok, ks * kBK,
                           tl.row0, fb);
             }
             ++issued;
@@ -312,10 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // exit drain: every token copy issued has landed.  `full` also counts converter
       // arrivals, so wait on the copies' own completion: the stage's phase can only
       // complete once its bytes are in (or the CTA aborted, which the drain bound covers).
-      if (lane == 0) {
-        if (PAIR) drain_ring(bar->tok_full, kTokStagesP, issued, err, 0x2F0);
-        else drain_ring(bar->full, kStages, issued, err, 0x2F0);
-      }
+      if (lane == 0) drain_ring(bar->full, kStages, issued, err, 0x2F0);
     } else if (warp == 2) {
       // ============================ weight + scale producer =========================
       int issued = 0, sc_issued = 0;
@@ -326,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t wph = 0;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
           Tile tl;
-          decode_tile<PAIR>(t, s_tstart, s_off, E, nfb, tl);
+          decode_tile(t, s_tstart, s_off, E, nfb, tl);
           const int rows = min(kBM, N - tl.feat0);
           const int sb = lt & 1;
           if (!mbar_wait_sleep(smem_u32(&bar->sc_empty[sb]), ((lt >> 1) & 1) ^ 1, err, 0x200, s_abort, 128)) break;
@@ -351,17 +298,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait_sleep(smem_u32(&bar->w_empty[ws]), wph ^ 1, err, 0x202, s_abort, 64)) { ok = false; break; }
             const uint32_t fb = smem_u32(&bar->w_full[ws]);
             mbar_arrive_expect_tx(fb, kWBytes);
-            tma_load_2d(smem_u32(smem + SL::w + ws * kWBytes), &tmap_w, ks * (kBK / 2),
+            tma_load_2d(smem_u32(smem + SmemLayout::w + ws * kWBytes), &tmap_w, ks * (kBK / 2),
                         tl.e * N + tl.feat0, fb);
             ++issued;
-            if (++ws == WST) { ws = 0; wph ^= 1; }
+            if (++ws == kWStages) { ws = 0; wph ^= 1; }
           }
         }
       }
       __syncwarp();
       __syncthreads();
       if (lane == 0) {
-        drain_ring(bar->w_full, WST, issued, err, 0x2F1);
+        drain_ring(bar->w_full, kWStages, issued, err, 0x2F1);
         drain_ring(bar->sc_full, 2, sc_issued, err, 0x2F2);
       }
     } else if (warp == 1) {
@@ -369,59 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         int s = 0;
         uint32_t ph = 0;
-        const uint32_t tok_base = smem_u32(smem + SL::tok);
+        const uint32_t tok_base = smem_u32(smem + SmemLayout::tok);
         int lt = 0;
         bool ok = true;
-        int ts = 0;  // paired form: token ring stage and phase
-        uint32_t tph = 0;
-        for (int t = blockIdx.x; t < total && ok && PAIR; t += gridDim.x, ++lt) {
-          // ---- paired form: every A stage feeds the MMAs of both sub-tiles ---------------
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
           Tile tl;
-          decode_tile<PAIR>(t, s_tstart, s_off, E, nfb, tl);
-          // one accumulator pair per tile: wait until the epilogue has drained the last tile
-          if (!mbar_wait(smem_u32(&bar->acc_empty[0]), (lt & 1) ^ 1, err, 0x300, s_abort)) break;
-          tc_fence_after();
-          const uint32_t idesc0 = idesc_bf16_m128((tl.n0 + 15) & ~15);
-          const uint32_t idesc1 = idesc_bf16_m128((tl.n1 + 15) & ~15);
-          for (int ks = 0; ks < nk && ok; ks += 2) {
-            const bool two = ks + 1 < nk;
-            const int s1 = (s + 1 == kStages) ? 0 : s + 1;
-            const uint32_t ph1 = (s + 1 == kStages) ? (ph ^ 1) : ph;
-            if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort) ||
-                (two && !mbar_wait(smem_u32(&bar->full[s1]), ph1, err, 0x301, s_abort))) {
-              ok = false;
-              break;
-            }
-            for (int h = 0; h < 2 && ok; ++h) {
-              if (h == 1 && !two) break;
-              const int st = h ? s1 : s;
-              const uint32_t a_tmem = tmem + kACol0 + st * (kBK / 2);
-              for (int j = 0; j < 2; ++j) {
-                if (j == 1 && tl.n1 == 0) break;
-                if (!mbar_wait(smem_u32(&bar->tok_full[ts]), tph, err, 0x302, s_abort)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-                const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + ts * kTokBytes);
-                const uint32_t d_tmem = tmem + j * kAccCols;
-#pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                  mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2),
-                              j ? idesc1 : idesc0, (ks | h | kk) != 0);
-                mma_commit(smem_u32(&bar->tok_empty[ts]));
-                if (++ts == kTokStagesP) { ts = 0; tph ^= 1; }
-              }
-              if (ok) mma_commit(smem_u32(&bar->empty[st]));
-            }
-            s = two ? ((s1 + 1 == kStages) ? 0 : s1 + 1) : s1;
-            ph = two ? ((s1 + 1 == kStages) ? (ph1 ^ 1) : ph1) : ph1;
-          }
-          if (ok) mma_commit(smem_u32(&bar->acc_full[0]));
-        }
-        for (int t = blockIdx.x; t < total && ok && !PAIR; t += gridDim.x, ++lt) {
-          Tile tl;
-          decode_tile<PAIR>(t, s_tstart, s_off, E, nfb, tl);
+          decode_tile(t, s_tstart, s_off, E, nfb, tl);
           const int acc = lt & 1;
           if (!mbar_wait(smem_u32(&bar->acc_empty[acc]), ((lt >> 1) & 1) ^ 1, err, 0x300, s_abort)) break;
           tc_fence_after();
@@ -508,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cidx = warp - 4;
     const int par = cidx >> 2;
     // per-warp scale-factor words (transposed scales): f1 of k-steps 0/1, then f2 of 0/1
-    uint32_t* cw = reinterpret_cast<uint32_t*>(smem + SL::cw) + cidx * 128;
+    uint32_t* cw = reinterpret_cast<uint32_t*>(smem + SmemLayout::cw) + cidx * 128;
     const int r = 32 * q + lane;  // row of the 128-row weight tile
     // 32B-swizzled packed tile: the two 16-byte halves of row r swap when bit 2 of r is set
     const int swz = (r >> 2) & 1;
@@ -519,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt, g += nk) {
       Tile tl;
-      decode_tile<PAIR>(t, s_tstart, s_off, E, nfb, tl);
+      decode_tile(t, s_tstart, s_off, E, nfb, tl);
       const bool active = tl.feat0 + 32 * q < N;  // warp-uniform: N % 32 == 0
       const int sb = lt & 1;
       if (!mbar_wait_sleep(smem_u32(&bar->sc_full[sb]), (lt >> 1) & 1, err, 0x400, s_abort, 64)) break;
@@ -577,15 +477,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           if (h == 1 && !two) break;
-          const int s = (ga + h) % WST;
-          if (!mbar_wait_sleep(smem_u32(&bar->w_full[s]), ((ga + h) / WST) & 1, err, 0x401,
+          const int s = (ga + h) % kWStages;
+          if (!mbar_wait_sleep(smem_u32(&bar->w_full[s]), ((ga + h) / kWStages) & 1, err, 0x401,
                          s_abort, 32)) {
             ok = false;
             break;
           }
           uint32_t qw[8];
           {
-            const uint8_t* row = smem + SL::w + s * kWBytes + r * (kBK / 2);
+            const uint8_t* row = smem + SmemLayout::w + s * kWBytes + r * (kBK / 2);
             const uint4 w0 = *reinterpret_cast<const uint4*>(row + (swz << 4));
             const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((swz ^ 1) << 4));
             qw[0] = w0.x; qw[1] = w0.y; qw[2] = w0.z; qw[3] = w0.w;
@@ -693,10 +593,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the A stages (this also orders the pair's reads of cw before the next pair's writes)
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(smem_u32(&bar->w_empty[ga % WST]));
+          mbar_arrive(smem_u32(&bar->w_empty[ga % kWStages]));
           mbar_arrive(smem_u32(&bar->full[ga % kStages]));
           if (two) {
-            mbar_arrive(smem_u32(&bar->w_empty[(ga + 1) % WST]));
+            mbar_arrive(smem_u32(&bar->w_empty[(ga + 1) % kWStages]));
             mbar_arrive(smem_u32(&bar->full[(ga + 1) % kStages]));
           }
         }
@@ -714,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
       Tile tl;
-      decode_tile<PAIR>(t, s_tstart, s_off, E, nfb, tl);
+      decode_tile(t, s_tstart, s_off, E, nfb, tl);
       const int acc = lt & 1;
       const int f = tl.feat0 + 32 * q + lane;  // output feature of this thread
       const bool active = tl.feat0 + 32 * q < N;
@@ -726,25 +626,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j)
           dnext[j] = __ldg(p.dgu + (size_t)min(tl.row0 + j, p.A - 1) * N + f);
       }
-      // paired form: one accumulator pair per tile (index 0), phase = tile parity
-      const int abar = PAIR ? 0 : acc;
-      const uint32_t aph = PAIR ? (uint32_t)(lt & 1) : (uint32_t)((lt >> 1) & 1);
-      if (!mbar_wait_sleep(smem_u32(&bar->acc_full[abar]), aph, err, 0x500, s_abort, 256)) break;
+      if (!mbar_wait_sleep(smem_u32(&bar->acc_full[acc]), (lt >> 1) & 1, err, 0x500, s_abort, 256)) break;
       tc_fence_after();
       float bias_f = 0.f;
       if ((EPI == kEpiGateUp || EPI == kEpiDown) && active)
         bias_f = bf16_to_f(p.bias[(size_t)tl.e * N + f]);
-      // 32-row chunks of sub-tile 0, then of sub-tile 1 (paired form), in row order
-      const int nch0 = (tl.n0 + 31) >> 5, nch = nch0 + ((tl.n1 + 31) >> 5);
-      for (int ci = 0; ci < nch; ++ci) {
-        const int sj = ci >= nch0 ? 1 : 0;
-        const int c0 = (ci - (sj ? nch0 : 0)) * 32;
+      for (int c0 = 0; c0 < tl.n_valid; c0 += 32) {
         uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (PAIR ? sj : acc) * kAccCols + c0, r);
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + acc * kAccCols + c0, r);
         tmem_wait_ld();
         if (!active) continue;
-        const int ncol = min(32, (sj ? tl.n1 : tl.n0) - c0);
-        const int rbase = tl.row0 + (sj ? tl.n0 : 0) + c0;
+        const int ncol = min(32, tl.n_valid - c0);
+        const int rbase = tl.row0 + c0;
         const bool odd = (lane & 1) != 0;
         if (EPI == kEpiGateUp) {
           // Columns j (even lane) and j+1 (odd lane) of each pair: the lanes of an
@@ -817,10 +710,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t dcur[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) dcur[j] = dnext[j];
-            if (ci + 1 < nch) {  // the next chunk's rows follow this one's in both forms
+            if (c0 + 32 < tl.n_valid) {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                dnext[j] = __ldg(p.dgu + (size_t)min(rbase + ncol + j, p.A - 1) * I + f);
+                dnext[j] = __ldg(p.dgu + (size_t)min(rbase + 32 + j, p.A - 1) * I + f);
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -833,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar->acc_empty[abar]));
+      if (lane == 0) mbar_arrive(smem_u32(&bar->acc_empty[acc]));
     }
     __syncwarp();
     __syncthreads();
@@ -865,10 +758,10 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int EPI, bool COLT, bool BS, bool PAIR>
+template <int EPI, bool COLT, bool BS>
 cudaError_t launch_one(const CUtensorMap& tt, const CUtensorMap& tl, const CUtensorMap& tw,
                        const GemmArgs& a, int grid, size_t smem, cudaStream_t st) {
-  auto kern = grouped_gemm_kernel<EPI, COLT, BS, PAIR>;
+  auto kern = grouped_gemm_kernel<EPI, COLT, BS>;
   // the setmaxnreg split assumes kLaunchRegs registers per thread at launch
   cudaFuncAttributes fa;
   cudaError_t fe = cudaFuncGetAttributes(&fa, kern);
@@ -894,17 +787,11 @@ bool encode_2d(EncodeTiledFn enc, CUtensorMap* m, CUtensorMapDataType type, cons
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t smem_bytes(bool pair, int K, int sfb_stride) {
-  const size_t sc = pair ? SmemLayoutT<true>::sc : SmemLayoutT<false>::sc;
-  return 1024 + sc + 2 * ((size_t)(4 * K) + (size_t)kBN * sfb_stride);
-}
-
-constexpr size_t kMaxSmem = 232448;  // 227 KB of opt-in dynamic shared memory per block
-
 }  // namespace
 
-// The bf16 (unpaired) form's size: the one every shape must fit.
-size_t grouped_gemm_smem_bytes(int K, int sfb_stride) { return smem_bytes(false, K, sfb_stride); }
+size_t grouped_gemm_smem_bytes(int K, int sfb_stride) {
+  return 1024 + SmemLayout::sc + 2 * ((size_t)(4 * K) + (size_t)kBN * sfb_stride);
+}
 
 cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const void* tokens,
                                 const uint8_t* wq, const GemmArgs& a, int num_sms,
@@ -931,27 +818,16 @@ cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const void* tok
   if (!encode_2d(enc, &tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, 1, a.K / 2,
                  (uint64_t)a.E * (uint64_t)a.N, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
+  const size_t smem = grouped_gemm_smem_bytes(a.K, bs ? a.sfb_stride : 0);
   const int grid = num_sms;
-  if (bs) {
-    const size_t smem = smem_bytes(false, a.K, a.sfb_stride);
-    return launch_one<kEpiGateUp, false, true, false>(tt, tl, tw, a, grid, smem, st);
-  }
-  // the paired form whenever its deeper token ring fits shared memory
-  const size_t smem_p = smem_bytes(true, a.K, 0);
-  const bool pair = smem_p <= kMaxSmem;
-  const size_t smem = pair ? smem_p : smem_bytes(false, a.K, 0);
-  switch ((epi * 2 + (transposed_scales ? 1 : 0)) * 2 + (pair ? 1 : 0)) {
-    case (kEpiGateUp * 2 + 0) * 2 + 0: return launch_one<kEpiGateUp, false, false, false>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiGateUp * 2 + 0) * 2 + 1: return launch_one<kEpiGateUp, false, false, true>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiDown * 2 + 0) * 2 + 0: return launch_one<kEpiDown, false, false, false>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiDown * 2 + 0) * 2 + 1: return launch_one<kEpiDown, false, false, true>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiDact * 2 + 1) * 2 + 0: return launch_one<kEpiDact, true, false, false>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiDact * 2 + 1) * 2 + 1: return launch_one<kEpiDact, true, false, true>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiDx * 2 + 1) * 2 + 0: return launch_one<kEpiDx, true, false, false>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiDx * 2 + 1) * 2 + 1: return launch_one<kEpiDx, true, false, true>(tt, tl, tw, a, grid, smem, st);
+  if (bs) return launch_one<kEpiGateUp, false, true>(tt, tl, tw, a, grid, smem, st);
+  switch (epi * 2 + (transposed_scales ? 1 : 0)) {
+    case kEpiGateUp * 2 + 0: return launch_one<kEpiGateUp, false, false>(tt, tl, tw, a, grid, smem, st);
+    case kEpiDown * 2 + 0: return launch_one<kEpiDown, false, false>(tt, tl, tw, a, grid, smem, st);
+    case kEpiDact * 2 + 1: return launch_one<kEpiDact, true, false>(tt, tl, tw, a, grid, smem, st);
+    case kEpiDx * 2 + 1: return launch_one<kEpiDx, true, false>(tt, tl, tw, a, grid, smem, st);
     // plain product over the stored rows (the grouped matmul entry point)
-    case (kEpiDx * 2 + 0) * 2 + 0: return launch_one<kEpiDx, false, false, false>(tt, tl, tw, a, grid, smem, st);
-    case (kEpiDx * 2 + 0) * 2 + 1: return launch_one<kEpiDx, false, false, true>(tt, tl, tw, a, grid, smem, st);
+    case kEpiDx * 2 + 0: return launch_one<kEpiDx, false, false>(tt, tl, tw, a, grid, smem, st);
     default: return cudaErrorInvalidValue;
   }
 }

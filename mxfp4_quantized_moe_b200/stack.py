@@ -49,8 +49,26 @@ def _wide(t: torch.Tensor) -> torch.Tensor:
 
 def router_logits(x: torch.Tensor, w_r: torch.Tensor, b_r: torch.Tensor) -> torch.Tensor:
     """Logits of the residual stream, x W_r + b_r (the caller's router linear), in fp32 for
-    a bf16 stream."""
+    a bf16 stream.  On the GPU a bf16 stream goes through one GEMM with fp32 accumulation and
+    fp32 output (no widened copy of x)."""
+    if x.is_cuda and x.dtype == torch.bfloat16 and w_r.dtype == torch.bfloat16:
+        return torch.addmm(_wide(b_r), x, w_r, out_dtype=torch.float32)
     return torch.addmm(_wide(b_r), _wide(x), _wide(w_r))
+
+
+def residual_add(x: torch.Tensor, y: torch.Tensor) -> torch.Tensor:
+    """x + y in fp32, rounded once to the stream's dtype (one elementwise kernel: torch adds
+    16-bit floats in fp32 and rounds the result)."""
+    return x + y if x.dtype == y.dtype else (_wide(x) + _wide(y)).to(x.dtype)
+
+
+def grad_chain(g: torch.Tensor, dx: torch.Tensor, d_logits: torch.Tensor,
+               w_r: torch.Tensor) -> torch.Tensor:
+    """g + dx + d_logits W_r^T in fp32, rounded once to g's dtype: the router path's GEMM
+    accumulates onto g (fp32), then dx is added in place."""
+    acc = torch.addmm(_wide(g), _wide(d_logits), _wide(w_r).t())
+    acc += dx
+    return acc.to(g.dtype)
 
 
 class MoeStack:
@@ -97,7 +115,7 @@ class MoeStack:
             y = self.block_forward(l, x, logits)
             if tap is not None:
                 tap(l, {"x": x, "logits": logits, "y": y})
-            x = (_wide(x) + _wide(y)).to(x.dtype)
+            x = residual_add(x, y)
         return x, saved
 
     def backward(self, dy: torch.Tensor, saved: list, tap: Callable | None = None):
@@ -113,7 +131,7 @@ class MoeStack:
             if tap is not None:
                 tap(l, {"g": g, "dx": dx_moe, "d_logits": d_logits,
                         "d_w": out[2] if len(out) > 2 else None})
-            g = (_wide(g) + _wide(dx_moe) + _wide(d_logits) @ _wide(b.w_r).t()).to(g.dtype)
+            g = grad_chain(g, dx_moe, d_logits, b.w_r)
         return g
 
 
