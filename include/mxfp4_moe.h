@@ -71,7 +71,8 @@ extern "C" {
 #define MXFP4_MOE_ERR_DEVICE_TIMEOUT (-5)       /* a bounded device-side wait expired      */
 #define MXFP4_MOE_ERR_DEVICE_BOUNDS (-6)        /* a device-side index check failed        */
 
-/* Problem shape and GLU constants (GPT-OSS: glu_alpha = 1.702, glu_limit = 7). */
+/* Problem shape and GLU constants (GPT-OSS: glu_alpha = 1.702, glu_limit = 7).
+ * Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", section "What this does" (the GptOssExperts expert loop and its activation). */
 typedef struct {
   int32_t T, H, I, E, k;
   float glu_alpha;
@@ -79,6 +80,8 @@ typedef struct {
 } mxfp4_moe_dims;
 
 /* Frozen expert weights in the packed MXFP4 layout (read only, never modified).
+ * Source: "Integrate finegrained kernels: SOTA performance and per-module quantization", the loader commit (`_blocks` / `_scales` tensors) and the gate|up row
+ * interleave commit; OCP Microscaling Formats (MX) v1.0 for the E2M1 / UE8M0 encodings.
  *   gu_blocks  uint8 [E][2I][H/2]  gate_up rows, interleaved: row 2j = gate j, row 2j+1 = up j.
  *                                  Byte i of a row holds element 2i (low nibble) and 2i+1
  *                                  (high nibble), E2M1 codes.
@@ -98,17 +101,20 @@ typedef struct {
   const uint16_t* dn_bias;
 } mxfp4_moe_weights;
 
-/* Bytes of device workspace that mxfp4_moe_forward / mxfp4_moe_backward_input need for `d`.
+/* Bytes of device workspace that mxfp4_moe_forward / mxfp4_moe_backward_input need for `d`
+ * (no counterpart in the pages: the caller-owned memory of this interface).
  * The forward leaves its saved state in the workspace (routing, permutation, the GLU output and
  * its two derivative factors per (assignment, feature)); the backward reads it and uses the
  * rest as scratch.
  * Errors: INVALID_ARG (null pointers, bad shape). */
 MXFP4_MOE_API int mxfp4_moe_workspace_size(const mxfp4_moe_dims* d, size_t* bytes);
 
-/* Bytes of the transposed weight copy made by mxfp4_moe_transpose_weights. */
+/* Bytes of the transposed weight copy made by mxfp4_moe_transpose_weights (no counterpart in
+ * the pages). */
 MXFP4_MOE_API int mxfp4_moe_transposed_weights_size(const mxfp4_moe_dims* d, size_t* bytes);
 
-/* One-time layout step for the backward (weights are frozen, so it is done once per set of
+/* One-time layout step for the backward (no counterpart in the pages; like "Integrate finegrained kernels: SOTA performance and per-module quantization"'s one-time
+ * post-load layout conversions).  Weights are frozen, so it is done once per set of
  * weights, not per step).  The input-gradient GEMMs contract over the OUTPUT axis of the
  * stored weights (dact = dy W_d, dx = dh W_gu), where the 32-element scale blocks run across
  * the contraction.  This call writes the same E2M1 codes and UE8M0 scale bytes, transposed:
@@ -122,7 +128,8 @@ MXFP4_MOE_API int mxfp4_moe_transposed_weights_size(const mxfp4_moe_dims* d, siz
 MXFP4_MOE_API int mxfp4_moe_transpose_weights(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, void* wt,
                                 size_t wt_bytes, void* stream);
 
-/* Forward.
+/* Forward.  Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", section "What this does" (top-k router + expert loop over weights
+ * dequantized on the fly); "Integrate finegrained kernels: SOTA performance and per-module quantization", commits on the gate|up interleave and the per-expert bias.
  *   x        bf16  [T][H]   activations
  *   logits   fp32  [T][E]   router logits (the router linear stays with the caller)
  *   y        bf16  [T][H]   output: sum_j w_{t,j} y_{t,j}
@@ -177,6 +184,8 @@ MXFP4_MOE_API int mxfp4_moe_forward_static(const mxfp4_moe_dims* d, const mxfp4_
 MXFP4_MOE_API int mxfp4_moe_forward_static_check(void* stream, int32_t* where);
 
 /* Input-gradient backward through the frozen quantized weights (no weight gradient).
+ * Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", sections "Why (the silent-gradient trap)" and "Relation to the backward
+ * triton kernels" (gradients must reach the inputs through the expert math).
  *   wt       the transposed copy from mxfp4_moe_transpose_weights for the same weights
  *   dy       bf16 [T][H]  upstream gradient dL/d(out)
  *   ws       the workspace the matching mxfp4_moe_forward used (its saved state is read; the
@@ -231,6 +240,7 @@ MXFP4_MOE_API int mxfp4_moe_grouped_matmul(int32_t E, int32_t N, int32_t K, int3
                                            void* stream);
 
 /* Standalone dequantization (diagnostics and tests): rows of packed MXFP4 -> bf16.
+ * Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", section "What this does" (`_dequantize_weights`); OCP MX v1.0.
  *   blocks uint8 [rows][K/2], scales uint8 [rows][K/32], out bf16 [rows][K]; K multiple of 32.
  * out = bf16(E2M1(code) * 2^(s-127)), exact (the product is always representable in bf16 or
  * overflows to inf); s = 255 gives NaN.
@@ -238,7 +248,8 @@ MXFP4_MOE_API int mxfp4_moe_grouped_matmul(int32_t E, int32_t N, int32_t K, int3
 MXFP4_MOE_API int mxfp4_moe_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
                          uint16_t* out, void* stream);
 
-/* Synchronize `stream`, then read and clear the device error word in `ws` (a workspace used by
+/* (No counterpart in the pages: failure detection of this library.)
+ * Synchronize `stream`, then read and clear the device error word in `ws` (a workspace used by
  * forward/backward).  Returns 0, DEVICE_TIMEOUT or DEVICE_BOUNDS (from the device), or CUDA
  * if the stream reported an error.  `where` (may be NULL) receives the device-side tag. */
 MXFP4_MOE_API int mxfp4_moe_check(void* ws, void* stream, int32_t* where);
@@ -257,7 +268,7 @@ MXFP4_MOE_API int mxfp4_moe_check(void* ws, void* stream, int32_t* where);
  * Errors: INVALID_ARG (null, short or misaligned ws), UNSUPPORTED_DEVICE, CUDA. */
 MXFP4_MOE_API int mxfp4_moe_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream);
 
-/* Per-kernel timing (diagnostics).  Between mxfp4_moe_profile_begin() and
+/* Per-kernel timing (diagnostics; no counterpart in the pages).  Between mxfp4_moe_profile_begin() and
  * mxfp4_moe_profile_end(), the library records a CUDA event pair on the launching stream around
  * every kernel it enqueues (host-side bookkeeping only; results are unchanged).
  * mxfp4_moe_profile_end synchronizes those events and fills up to `max` entries of `out` with
@@ -272,7 +283,7 @@ typedef struct {
 MXFP4_MOE_API int mxfp4_moe_profile_begin(void);
 MXFP4_MOE_API int mxfp4_moe_profile_end(mxfp4_moe_kernel_time* out, int32_t max, int32_t* n);
 
-/* Static description of a return code. */
+/* Static description of a return code (no counterpart in the pages). */
 MXFP4_MOE_API const char* mxfp4_moe_strerror(int code);
 
 #ifdef __cplusplus
