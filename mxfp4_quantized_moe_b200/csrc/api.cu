@@ -21,8 +21,9 @@ struct WsLayout {
 };
 
 // Row stride of the activation scales the block-scaled gate_up GEMM reads: one byte per
-// 32 elements of H, padded to whole k-steps (two blocks each) and to 16 bytes (bulk copies).
-int sfb_stride(int H) { return (2 * ((H + moe::kBK - 1) / moe::kBK) + 15) / 16 * 16; }
+// 32 elements of H, padded to whole k-steps (two blocks each) and to 32 bytes (bulk copies
+// want 16; the bank swizzle of the scale words exchanges words within 32-byte groups).
+int sfb_stride(int H) { return (2 * ((H + moe::kBK - 1) / moe::kBK) + 31) / 32 * 32; }
 
 // Workspace regions, each 256-byte aligned, in this order.  The forward leaves the routing
 // (idx, w, perm, inv, w_row), the GLU derivative factors (dgu) and the expert outputs y in

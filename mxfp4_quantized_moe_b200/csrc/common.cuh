@@ -288,6 +288,38 @@ MOE_DEV float fast_sigmoid(float z) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
   return fmaf(0.5f, t, 0.5f);
 }
+// Two fp32 values in one 64-bit register for the paired fp32 arithmetic of sm_100
+// (add / mul / fma .f32x2: one instruction for both lanes of the pair).
+MOE_DEV uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+MOE_DEV float f2lo(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+MOE_DEV float f2hi(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+MOE_DEV uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+MOE_DEV uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+MOE_DEV uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 MOE_DEV uint32_t pack_bf16x2(float lo, float hi) {
   return (uint32_t)f_to_bf16(lo) | ((uint32_t)f_to_bf16(hi) << 16);
 }

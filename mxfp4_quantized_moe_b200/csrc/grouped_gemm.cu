@@ -48,6 +48,8 @@ namespace {
 // MMA-facing ring: stage s holds the token tile (shared memory) and the bf16 A operand
 // (TMEM) of one k-step; the MMA waits once and commits once per k-step.
 constexpr int kStages = 4;        // even: a stage always belongs to the same converter parity
+// Publish and issue each k-step on its own (true) or the two k-steps of a pair together (false).
+constexpr bool kStageIssue = true;
 constexpr int kWStages = 8;       // packed-weight ring depth (even, same reason)
 constexpr int kThreads = 512;
 constexpr int kConvWarps = 8;
@@ -327,6 +329,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t idesc = idesc_bf16_m128((tl.n_valid + 15) & ~15);
           const uint32_t d_tmem = tmem + acc * kAccCols;
+          if (kStageIssue) {
+            // one k-step per round: wait for its stage, issue its MMAs, release it on completion
+            const int npad = (tl.n_valid + 15) & ~15;
+            for (int ks = 0; ks < nk; ++ks) {
+              if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t tbase = tok_base + s * kTokBytes;
+              if (BS) {
+                const uint64_t bhi = smem_desc_kmajor_sw64(tbase);
+                const uint64_t blo = smem_desc_kmajor_sw64(tbase + kTokBytes / 2);
+                const uint32_t a_tmem = tmem + kACol0 + s * kAColsBS;
+                const uint32_t sfa = tmem + kSfaCol0 + s * 4, sfb = tmem + kSfbCol0 + s * 8;
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                  const uint32_t id = idesc_mxf4a_m128(npad, (uint32_t)kk);
+                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, bhi + (uint64_t)(kk * 2), id, sfa, sfb,
+                              (ks | kk) != 0);
+                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, blo + (uint64_t)(kk * 2), id, sfa, sfb, 1u);
+                }
+              } else {
+                const uint64_t bdesc = smem_desc_kmajor_sw128(tbase);
+                const uint32_t a_tmem = tmem + kACol0 + s * (kBK / 2);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                  mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
+                              (ks | kk) != 0);
+              }
+              mma_commit(smem_u32(&bar->empty[s]));
+              if (++s == kStages) { s = 0; ph ^= 1; }
+            }
+            if (ok) mma_commit(smem_u32(&bar->acc_full[acc]));
+            continue;
+          }
           // Two k-steps per round: both stages are waited for first, then their eight MMAs
           // go out back to back (the issuing thread blocks while the tensor pipe is busy, so
           // the bookkeeping between rounds is the only gap the pipe can see).
@@ -434,8 +472,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // re-derived from the scale bytes where it is needed)
         uint32_t f1[4] = {0, 0, 0, 0};
         bool slow = false;
+        // block-scaled form: the token tile's activation scales of the pair's four 32-element
+        // blocks, one 32-bit word per token (word u of the token's row, stored at word
+        // u ^ ((row / 4) % 8) so that the 32 lanes' loads hit 32 different banks)
+        uint32_t sfb4[kSfbCols];
         if (BS) {
           // the block-scaled MMA applies the UE8M0 scales itself (scale-factor columns)
+          const uint8_t* sfbb = scb + 4 * K;
+#pragma unroll
+          for (int j = 0; j < kSfbCols; ++j) {
+            const int tok = 32 * j + lane;
+            const int wsw = u ^ (((tl.row0 + tok) >> 2) & 7);
+            sfb4[j] = tok < tl.n_valid
+                          ? *reinterpret_cast<const uint32_t*>(sfbb + tok * p.sfb_stride + 4 * wsw)
+                          : 0u;
+          }
         } else if (!COLT) {
           uint32_t mx = 0;
 #pragma unroll
@@ -474,6 +525,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // each k-step: wait for its packed bytes, expand them to bf16 in registers, wait for
         // its A stage to be free (the MMA consumed the k-step kStages earlier) and store it
         const uint32_t lanes = (uint32_t)(32 * q) << 16;
+        // k-step j converted and stored: release its packed bytes and publish its A stage
+        // (the warp's reads of cw for it are ordered before any later write by the syncwarp)
+        auto publish_stage = [&](int j, bool stored) {
+          if (stored) tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&bar->w_empty[j % kWStages]));
+            mbar_arrive(smem_u32(&bar->full[j % kStages]));
+          }
+        };
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           if (h == 1 && !two) break;
@@ -510,15 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t b1 = (rv && blk0 + 1 < kb32) ? scb[r * kb32 + blk0 + 1] : 0u;
               sfa1 = b0 | (b1 << 8);
             }
-            const uint8_t* sfbb = scb + 4 * K;
             uint32_t sfb8[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int tok = 32 * j + lane;
-              sfb8[j] = (j < kSfbCols && tok < tl.n_valid)
-                            ? *reinterpret_cast<const uint16_t*>(sfbb + tok * p.sfb_stride + blk0)
-                            : 0u;
-            }
+            for (int j = 0; j < 8; ++j) sfb8[j] = j < kSfbCols ? (h ? sfb4[j] >> 16 : sfb4[j] & 0xFFFFu) : 0u;
             const int sa = (ga + h) % kStages;
             if (!mbar_wait(smem_u32(&bar->empty[sa]), (((ga + h) / kStages) & 1) ^ 1, err, 0x402,
                            s_abort)) {
@@ -529,6 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (active) tmem_st16(tmem + lanes + kACol0 + sa * kAColsBS, out16);
             tmem_st1(tmem + lanes + kSfaCol0 + sa * 4 + q, sfa1);
             tmem_st8(tmem + lanes + kSfbCol0 + sa * 8, sfb8);
+            if (kStageIssue) publish_stage(ga + h, true);
             continue;
           }
           uint32_t out[32];
@@ -585,8 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           if (active) tmem_st32(tmem + lanes + kACol0 + sa * (kBK / 2), out);
+          if (kStageIssue) publish_stage(ga + h, active);
         }
         if (!ok) break;
+        if (kStageIssue) continue;
         if (active || BS) tmem_wait_st();
         tc_fence_before();
         // packed bytes consumed and A stages written: release the weight stages and publish
@@ -649,23 +708,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int jf = f >> 1;
           uint32_t dw16[16];
           float av[16];
+          // two columns per step with the paired fp32 instructions (same operations and
+          // rounding as one column at a time)
+          const uint64_t kBias = f2(bias_f, bias_f), kOne = f2(1.f, 1.f);
+          const uint64_t kHalfAlpha = f2(0.5f * p.alpha, 0.5f * p.alpha);
+          const uint64_t kHalf = f2(0.5f, 0.5f), kAlpha = f2(p.alpha, p.alpha);
+          const uint64_t kMinusOne = f2(-1.f, -1.f);
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const float v0 = __uint_as_float(r[2 * jj]) + bias_f;
-            const float v1 = __uint_as_float(r[2 * jj + 1]) + bias_f;
-            const float recv = __shfl_xor_sync(kFull, odd ? v0 : v1, 1);
-            const float g = odd ? recv : v0;
-            const float u = odd ? v1 : recv;
-            const float gc = fminf(g, p.limit);
-            const float uc = fminf(fmaxf(u, -p.limit), p.limit);
-            const float sg = fast_sigmoid(p.alpha * gc);
-            const float t1 = gc * sg;
-            const float up1 = uc + 1.f;
-            av[jj] = up1 * t1;
+          for (int jj = 0; jj < 16; jj += 2) {
+            const uint64_t va = f2add(f2(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 2])), kBias);
+            const uint64_t vb = f2add(f2(__uint_as_float(r[2 * jj + 1]), __uint_as_float(r[2 * jj + 3])), kBias);
+            const float v0a = f2lo(va), v0b = f2hi(va), v1a = f2lo(vb), v1b = f2hi(vb);
+            const float ra = __shfl_xor_sync(kFull, odd ? v0a : v1a, 1);
+            const float rb = __shfl_xor_sync(kFull, odd ? v0b : v1b, 1);
+            const float ga = odd ? ra : v0a, ua = odd ? v1a : ra;
+            const float gb = odd ? rb : v0b, ub = odd ? v1b : rb;
+            const uint64_t gc = f2(fminf(ga, p.limit), fminf(gb, p.limit));
+            const uint64_t uc = f2(fminf(fmaxf(ua, -p.limit), p.limit), fminf(fmaxf(ub, -p.limit), p.limit));
+            // sigmoid(a g') = (1 + tanh(a g' / 2)) / 2
+            const uint64_t z = f2mul(kHalfAlpha, gc);
+            float ta, tb;
+            asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(f2lo(z)));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(f2hi(z)));
+            const uint64_t sg = f2fma(kHalf, f2(ta, tb), kHalf);
+            const uint64_t t1 = f2mul(gc, sg);
+            const uint64_t up1 = f2add(uc, kOne);
+            const uint64_t act = f2mul(up1, t1);
+            av[jj] = f2lo(act);
+            av[jj + 1] = f2hi(act);
+            // d act / d g' = (u'+1) (s + a t1 (1 - s)); d act / d u' = t1
+            const uint64_t om = f2fma(sg, kMinusOne, kOne);
+            const uint64_t dg = f2mul(up1, f2fma(f2mul(kAlpha, t1), om, sg));
             // bf16(g) <= limit  <=>  g <= mask_limit (and likewise for |bf16(u)|)
-            const float dgc = (g <= p.mask_limit) ? up1 * (sg + p.alpha * t1 * (1.f - sg)) : 0.f;
-            const float duc = (fabsf(u) <= p.mask_limit) ? t1 : 0.f;
-            dw16[jj] = pack_bf16x2(dgc, duc);
+            const float dga = (ga <= p.mask_limit) ? f2lo(dg) : 0.f;
+            const float dgb = (gb <= p.mask_limit) ? f2hi(dg) : 0.f;
+            const float dua = (fabsf(ua) <= p.mask_limit) ? f2lo(t1) : 0.f;
+            const float dub = (fabsf(ub) <= p.mask_limit) ? f2hi(t1) : 0.f;
+            dw16[jj] = pack_bf16x2(dga, dua);
+            dw16[jj + 1] = pack_bf16x2(dgb, dub);
           }
           uint32_t* dgu_out = reinterpret_cast<uint32_t*>(p.out0);
 #pragma unroll
@@ -801,7 +881,7 @@ cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const void* tok
   const bool bs = a.tok_lo != nullptr;
   CUtensorMap tt, tl, tw;
   if (bs) {  // E4M3 hi / lo parts: [A][K] bytes each, 64-byte rows per k-step
-    if (epi != kEpiGateUp || transposed_scales || !a.sfb || a.sfb_stride % 16 ||
+    if (epi != kEpiGateUp || transposed_scales || !a.sfb || a.sfb_stride % 32 ||
         a.sfb_stride < 2 * ((a.K + kBK - 1) / kBK))
       return cudaErrorInvalidValue;
     if (!encode_2d(enc, &tt, CU_TENSOR_MAP_DATA_TYPE_UINT8, tokens, 1, a.K, a.A, kBK, kBN,

@@ -63,7 +63,8 @@ cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, 
 cudaError_t launch_gather_rows(const uint16_t* src, int H, int k, const int32_t* perm, int A,
                                uint16_t* dst, float* dot_w, cudaStream_t st);
 // Gather x into expert-sorted rows as two E4M3 parts with a UE8M0 scale per 32 elements
-// (hi, lo [A][H] bytes; sfb [A][sfb_stride] UE8M0 bytes).
+// (hi, lo [A][H] bytes; sfb [A][sfb_stride] UE8M0 bytes, sfb_stride a multiple of 32; byte b
+// of row r at word (b / 4) ^ ((r / 4) % 8), byte b % 4).
 cudaError_t launch_gather_quant(const uint16_t* x, int H, int k, const int32_t* perm, int A,
                                 uint8_t* hi, uint8_t* lo, uint8_t* sfb, int sfb_stride,
                                 cudaStream_t st);

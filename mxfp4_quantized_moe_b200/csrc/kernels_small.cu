@@ -303,9 +303,15 @@ __global__ void gather_quant_kernel(const uint16_t* __restrict__ x, int H, int k
   const int t = perm[row] / k;
   const int nb = H / 32;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+  // scale byte b of the row lives in 32-bit word (b / 4) ^ ((row / 4) % 8), byte b % 4: the
+  // GEMM's converter lanes read one word of 32 consecutive rows and so hit 32 different banks
+  // (the stride is a multiple of 32 bytes, so the exchange stays inside the row)
+  uint8_t* srow = sfb + (size_t)row * sfb_stride;
+  const int rsw = (row >> 2) & 7;
   for (int b = lane; b < sfb_stride; b += 32) {
+    const int pos = 4 * ((b >> 2) ^ rsw) + (b & 3);
     if (b >= nb) {
-      sfb[(size_t)row * sfb_stride + b] = 0;
+      srow[pos] = 0;
       continue;
     }
     uint32_t v[16];
@@ -348,7 +354,7 @@ __global__ void gather_quant_kernel(const uint16_t* __restrict__ x, int H, int k
     dh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
     dl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     dl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
-    sfb[(size_t)row * sfb_stride + b] = (uint8_t)sbyte;
+    srow[pos] = (uint8_t)sbyte;
   }
 }
 

@@ -208,6 +208,15 @@ def test_edge_cases(moe, T, H, I, E, k, seed, kw):
     check_all(got, ref)
 
 
+@pytest.mark.parametrize("T", [1, 64, 256])
+def test_small_token_gpt_oss_20b_every_token(moe, T):
+    """The small-token (decode-sized) batches of the gpt-oss-20b layer (H=I=2880, E=32, k=4),
+    every token checked: a handful of rows per expert, most experts with a single token tile
+    far below the tile height."""
+    got, ref = run_block(moe, T, 2880, 2880, 32, 4, seed=40 + T)
+    check_all(got, ref)
+
+
 def test_expert_gradient_is_not_silent(moe):
     """The pages' silent-gradient trap: dX must carry the expert path (not be zero)."""
     got, ref = run_block(moe, 16, 64, 64, 4, 2, seed=12)
@@ -318,8 +327,18 @@ def test_interleave_helper_restores_the_shipped_row_order(moe):
 
 def _sfb_stride(H):
     """Row stride of the activation scales: one byte per 32 elements, padded to whole 64-element
-    k-steps and to 16 bytes."""
-    return (2 * (-(-H // 64)) + 15) // 16 * 16
+    k-steps and to 32 bytes."""
+    return (2 * (-(-H // 64)) + 31) // 32 * 32
+
+
+def _sfb_natural(sfb):
+    """The activation scales in block order: the library stores byte b of row r in 32-bit word
+    (b // 4) ^ ((r // 4) % 8), byte b % 4."""
+    A, st = sfb.shape
+    b = np.arange(st)
+    r = np.arange(A)[:, None]
+    pos = 4 * ((b[None, :] >> 2) ^ ((r >> 2) & 7)) + (b[None, :] & 3)
+    return np.take_along_axis(sfb, pos, axis=1)
 
 
 def _ws_offsets(T, E, k, H=None, I=None):
@@ -371,7 +390,7 @@ def test_activation_split_matches_the_mx_definition(moe):
     hi = wsn[o["dh"]:o["dh"] + A * H].reshape(A, H)  # the forward leaves them in the dH region
     lo = wsn[o["dh"] + A * H:o["dh"] + 2 * A * H].reshape(A, H)
     st = _sfb_stride(H)
-    sfb = wsn[o["sfb"]:o["sfb"] + A * st].reshape(A, st)
+    sfb = _sfb_natural(wsn[o["sfb"]:o["sfb"] + A * st].reshape(A, st))
     xs = O.bf16_bits_to_f64(x.view(torch.int16).numpy().view(np.uint16))[perm // k]
     rhi, rlo, S = O.mx_split(xs)
     S = S.reshape(A, H // 32)
