@@ -59,7 +59,13 @@ def peaks():
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a grouped GEMM,
 # from an ncu capture of this bench's workload; summaries under profiles/.  An entry counts
 # only while the kernel's sources hash to `sources`: after any change it reads as null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/launch_list_gpt-oss-20b-moe-T8192.md (one launch of each after three warm-up steps)
+    ("gemm_gate_up_glu", "gpt-oss-20b-moe-T8192"): {"bytes": 474569216 + 526212608, "sources": "ccca7f1b0a5f61f0"},
+    ("gemm_down", "gpt-oss-20b-moe-T8192"): {"bytes": 330117888 + 159798016, "sources": "ccca7f1b0a5f61f0"},
+    ("gemm_dact_glu_bwd", "gpt-oss-20b-moe-T8192"): {"bytes": 712381696 + 345076224, "sources": "ccca7f1b0a5f61f0"},
+    ("gemm_dx", "gpt-oss-20b-moe-T8192"): {"bytes": 692749312 + 172007936, "sources": "ccca7f1b0a5f61f0"},
+}
 KERNEL_SOURCES = ("mxfp4_quantized_moe_b200/csrc/grouped_gemm.cu",
                   "mxfp4_quantized_moe_b200/csrc/common.cuh",
                   "mxfp4_quantized_moe_b200/csrc/kernels.h")

@@ -5,9 +5,11 @@
 * standalone dequantization (`mxfp4_moe_dequantize`) of a whole gpt-oss-20b gate_up weight
   set, E*2I rows of H elements: 0.5 B of codes + 1/32 B of scale read and 2 B of bf16 written
   per element;
-* the routing gather (`gather_x`: A rows of H bf16 read and written) and the combine
-  (`combine_y`: A rows read, T rows written) of one gpt-oss-20b layer step at T=8192, from
-  the library's per-kernel event timing.
+* the memory-bound kernels of one gpt-oss-20b layer step at T=8192, from the library's
+  per-kernel event timing: the forward gather with the MX split (`gather_x_mx`: A rows of H
+  bf16 read, the E4M3 hi and lo parts and one scale byte per 32 written), the combines
+  (`combine_y`, `combine_dx`: A rows read, T rows written) and the dY gather with the
+  routing-weight dot (`gather_dy_dw`: A rows of dY and of y read, A rows written).
 
 Prints one JSON line per stage with its algorithmic bytes, time and GB/s against the HBM copy
 bandwidth in MEASURED_PEAKS.json (or the fallback figure).
@@ -65,21 +67,29 @@ def main():
     del out, blocks, scales
     torch.cuda.empty_cache()
 
-    # ---- gather and combine of a layer step ---------------------------------------------
+    # ---- gathers and combines of a layer step ------------------------------------------
     shape = moe.MoeShape(wl.T, wl.H, wl.I, wl.E, wl.k)
     w = moe.weights_to(inp, dev)
-    x, lg = inp["x"].to(dev), inp["logits"].to(dev)
+    wt = moe.transpose_weights(shape, w)
+    x, lg, dy = inp["x"].to(dev), inp["logits"].to(dev), inp["dy"].to(dev)
     ws = moe.alloc_workspace(shape, dev)
     y = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
     for _ in range(3):
         moe.forward(shape, w, x, lg, ws, y=y)
+        moe.backward_input(shape, w, wt, dy, ws)
     torch.cuda.synchronize()
     moe.profile_begin()
     for _ in range(args.iters):
         moe.forward(shape, w, x, lg, ws, y=y)
+        moe.backward_input(shape, w, wt, dy, ws)
     kt = moe.profile_end()
-    A = wl.T * wl.k
-    for name, nbytes in (("gather_x", 2.0 * A * wl.H * 2), ("combine_y", (A + wl.T) * wl.H * 2.0)):
+    A, T, H = wl.T * wl.k, wl.T, wl.H
+    sfb_stride = (2 * (-(-H // 64)) + 31) // 32 * 32
+    stages = (("gather_x_mx", A * H * 2.0 + A * H * 2.0 + A * sfb_stride),
+              ("combine_y", (A + T) * H * 2.0),
+              ("gather_dy_dw", A * H * 2.0 * 3 + A * 4.0),
+              ("combine_dx", (A + T) * H * 2.0))
+    for name, nbytes in stages:
         launches, tot = kt[name]
         ms = tot / launches
         print(json.dumps({"stage": name, "bytes": nbytes, "ms": ms,
