@@ -286,6 +286,14 @@ MXFP4_MOE_API int mxfp4_moe_profile_end(mxfp4_moe_kernel_time* out, int32_t max,
 /* Static description of a return code (no counterpart in the pages). */
 MXFP4_MOE_API const char* mxfp4_moe_strerror(int code);
 
+/* How this library was built (no counterpart in the pages): bit 0 set for the debug build
+ * (libmxfp4_moe_debug.so, compiled with MXFP4_MOE_DEBUG=1), whose kernels check the indices
+ * they read from the workspace (perm, inv, the expert offsets) and record
+ * MXFP4_MOE_ERR_DEVICE_BOUNDS with a tag in the error word instead of making an access
+ * through a bad index.  The release build returns 0 and carries no such checks.  Never fails. */
+#define MXFP4_MOE_BUILD_DEBUG 1
+MXFP4_MOE_API int mxfp4_moe_build_flags(void);
+
 #ifdef __cplusplus
 }
 #endif

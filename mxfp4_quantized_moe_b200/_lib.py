@@ -11,7 +11,11 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmxfp4_moe.so")
+# MXFP4_MOE_LIBRARY=debug loads the debug build (device-side index checks), else the library
+_VARIANT = os.environ.get("MXFP4_MOE_LIBRARY", "")
+if _VARIANT not in ("", "release", "debug"):
+    raise RuntimeError(f"MXFP4_MOE_LIBRARY={_VARIANT!r}: expected 'debug' or 'release'")
+LIB_PATH = os.path.join(HERE, "libmxfp4_moe_debug.so" if _VARIANT == "debug" else "libmxfp4_moe.so")
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -66,6 +70,7 @@ SIGNATURES = {
     "mxfp4_moe_profile_end": (ctypes.c_int, [ctypes.POINTER(KernelTime), ctypes.c_int32,
                                              ctypes.POINTER(ctypes.c_int32)]),
     "mxfp4_moe_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "mxfp4_moe_build_flags": (ctypes.c_int, []),
 }
 
 

@@ -262,7 +262,7 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
   uint8_t* xhi = at<uint8_t>(ws, L.dh);
   uint8_t* xlo = xhi + (size_t)A * H;
   uint8_t* sfb = at<uint8_t>(ws, L.sfb);
-  MOE_LAUNCH("gather_x_mx", moe::launch_gather_quant(x, H, k, perm, A, xhi, xlo, sfb, sfb_stride(H), st));
+  MOE_LAUNCH("gather_x_mx", moe::launch_gather_quant(x, H, k, perm, A, xhi, xlo, sfb, sfb_stride(H), err, st));
 
   moe::GemmArgs g{};
   g.off = off; g.E = E; g.A = A; g.err = err;
@@ -277,7 +277,7 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
   g.scales = w->dn_scales; g.K = I; g.N = H; g.bias = w->dn_bias; g.out0 = rows; g.out1 = nullptr;
   MOE_LAUNCH("gemm_down", moe::launch_grouped_gemm(moe::kEpiDown, false, act, w->dn_blocks, g, sms, st));
   // out_t = sum_j w_{t,j} y_{t,j}
-  MOE_LAUNCH("combine_y", moe::launch_combine(rows, inv, wr, T, k, H, y, st));
+  MOE_LAUNCH("combine_y", moe::launch_combine(rows, inv, wr, T, k, H, y, err, st));
   return MXFP4_MOE_OK;
 }
 
@@ -313,7 +313,7 @@ int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w
   uint16_t* rows = at<uint16_t>(ws, L.rows);
 
   // d_topk_w[slot] = <dY_t, y_r> with the forward's y_r read in place, then dYp[r] = dY[t(r)]
-  MOE_LAUNCH("gather_dy_dw", moe::launch_gather_rows(dy, H, k, perm, A, rows, d_topk_w, st));
+  MOE_LAUNCH("gather_dy_dw", moe::launch_gather_rows(dy, H, k, perm, A, rows, d_topk_w, err, st));
   moe::GemmArgs g{};
   g.off = off; g.E = E; g.A = A; g.err = err;
   g.alpha = d->glu_alpha; g.limit = d->glu_limit;
@@ -323,7 +323,7 @@ int mxfp4_moe_backward_input(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w
   // dx = dH W_gu (contract over the 2I interleaved rows), per sorted row
   g.scales = at<uint8_t>(wtp, LT.gu_scales); g.K = 2 * I; g.N = H; g.out0 = rows; g.dgu = nullptr; g.w_row = nullptr;
   MOE_LAUNCH("gemm_dx", moe::launch_grouped_gemm(moe::kEpiDx, true, dh, at<uint8_t>(wtp, LT.gu_blocks), g, sms, st));
-  MOE_LAUNCH("combine_dx", moe::launch_combine(rows, inv, nullptr, T, k, H, dx, st));
+  MOE_LAUNCH("combine_dx", moe::launch_combine(rows, inv, nullptr, T, k, H, dx, err, st));
   MOE_LAUNCH("router_backward", moe::launch_router_backward(idx, wr, d_topk_w, T, E, k, d_logits, st));
   return MXFP4_MOE_OK;
 }
@@ -431,6 +431,8 @@ int mxfp4_moe_profile_end(mxfp4_moe_kernel_time* out, int32_t max, int32_t* n) {
   *n = cnt;
   return rc;
 }
+
+int mxfp4_moe_build_flags(void) { return MXFP4_MOE_DEBUG ? MXFP4_MOE_BUILD_DEBUG : 0; }
 
 const char* mxfp4_moe_strerror(int code) {
   switch (code) {

@@ -16,6 +16,13 @@
 
 namespace moe {
 
+// Debug build (-DMXFP4_MOE_DEBUG=1, libmxfp4_moe_debug.so): kernels also check the indices
+// they read from the workspace and record MXFP4_MOE_ERR_DEVICE_BOUNDS with a tag instead of
+// making the access.  The release build compiles those checks out.
+#ifndef MXFP4_MOE_DEBUG
+#define MXFP4_MOE_DEBUG 0
+#endif
+
 // ------------------------------------------------------------------ error word --------
 // err[0]: first error code (MXFP4_MOE_ERR_*), err[1]: where (kernel-specific tag).
 struct DevErr {
@@ -295,16 +302,8 @@ MOE_DEV uint64_t f2(float lo, float hi) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
   return r;
 }
-MOE_DEV float f2lo(uint64_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-MOE_DEV float f2hi(uint64_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
-}
+MOE_DEV float f2lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+MOE_DEV float f2hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
 MOE_DEV uint64_t f2add(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));

@@ -214,9 +214,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0;
+    bool bad = MXFP4_MOE_DEBUG && s_off[0] != 0;
     for (int e = 0; e < E; ++e) {
       s_tstart[e] = acc;
+      if (MXFP4_MOE_DEBUG && (s_off[e + 1] < s_off[e] || s_off[e + 1] > p.A)) bad = true;
       acc += token_tiles(s_off[e + 1] - s_off[e]) * nfb;
+    }
+    if (bad) {  // debug build: offsets that do not partition [0, A) -> no tiles at all
+      err.set(MXFP4_MOE_ERR_DEVICE_BOUNDS, 0x600);
+      for (int e = 0; e < E; ++e) s_tstart[e] = 0;
+      acc = 0;
     }
     s_tstart[E] = acc;
   }
@@ -664,7 +671,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar->sc_empty[sb]));
     }
+    // an aborted pair may leave TMEM stores in flight: none may outlive the allocation
     __syncwarp();
+    tmem_wait_st();
     __syncthreads();
   } else {
     // ================================ epilogue ======================================

@@ -6,6 +6,11 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+// 1 in the debug build (libmxfp4_moe_debug.so): kernels check workspace indices (common.cuh)
+#ifndef MXFP4_MOE_DEBUG
+#define MXFP4_MOE_DEBUG 0
+#endif
+
 namespace moe {
 
 // Tile shape of the grouped GEMMs: 128 weight rows (output features) in TMEM as the
@@ -61,16 +66,18 @@ cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, 
 // gather of dY), `dst` first holds the forward's expert outputs y in sorted order, which are
 // read in place: dot_w[perm[r]] = <src[perm[r] / k], y[r]> before the row is overwritten.
 cudaError_t launch_gather_rows(const uint16_t* src, int H, int k, const int32_t* perm, int A,
-                               uint16_t* dst, float* dot_w, cudaStream_t st);
+                               uint16_t* dst, float* dot_w, int* err, cudaStream_t st);
 // Gather x into expert-sorted rows as two E4M3 parts with a UE8M0 scale per 32 elements
 // (hi, lo [A][H] bytes; sfb [A][sfb_stride] UE8M0 bytes, sfb_stride a multiple of 32; byte b
 // of row r at word (b / 4) ^ ((r / 4) % 8), byte b % 4).
 cudaError_t launch_gather_quant(const uint16_t* x, int H, int k, const int32_t* perm, int A,
                                 uint8_t* hi, uint8_t* lo, uint8_t* sfb, int sfb_stride,
-                                cudaStream_t st);
+                                int* err, cudaStream_t st);
 // out[t] = sum_j w[t*k+j] * rows[inv[t*k+j]] in fp32, rounded to bf16 once (w == nullptr: 1).
+// `err` is the workspace error word: the debug build records out-of-range perm / inv entries
+// there (DEVICE_BOUNDS) instead of reading through them.
 cudaError_t launch_combine(const uint16_t* rows, const int32_t* inv, const float* w, int T, int k,
-                           int H, uint16_t* out, cudaStream_t st);
+                           int H, uint16_t* out, int* err, cudaStream_t st);
 // d_logits from d_topk_w through the softmax over the k selected logits (one thread per token)
 cudaError_t launch_router_backward(const int32_t* idx, const float* w, const float* d_topk_w,
                                    int T, int E, int k, float* d_logits, cudaStream_t st);

@@ -225,12 +225,16 @@ __device__ __forceinline__ float bf16x8_dot(const uint4& a, const uint4& b) {
 
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ src, int H, int k,
                                    const int32_t* __restrict__ perm, int A, uint16_t* dst,
-                                   float* __restrict__ dot_w) {
+                                   float* __restrict__ dot_w, int* err) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= A) return;
   const int row = warp;
   const int slot = perm[row];
+  if (MXFP4_MOE_DEBUG && (slot < 0 || slot >= A)) {  // warp-uniform
+    if (lane == 0) DevErr{err}.set(MXFP4_MOE_ERR_DEVICE_BOUNDS, 0x110);
+    return;
+  }
   const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(slot / k) * H);
   uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * H);
   const int nv = H / 8;
@@ -295,11 +299,15 @@ __device__ __forceinline__ void f32x2_from_e4m3x2(uint32_t v, float& lo, float& 
 __global__ void gather_quant_kernel(const uint16_t* __restrict__ x, int H, int k,
                                     const int32_t* __restrict__ perm, int A,
                                     uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
-                                    uint8_t* __restrict__ sfb, int sfb_stride) {
+                                    uint8_t* __restrict__ sfb, int sfb_stride, int* err) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= A) return;
   const int row = warp;
+  if (MXFP4_MOE_DEBUG && (perm[row] < 0 || perm[row] >= A)) {  // warp-uniform
+    if (lane == 0) DevErr{err}.set(MXFP4_MOE_ERR_DEVICE_BOUNDS, 0x111);
+    return;
+  }
   const int t = perm[row] / k;
   const int nb = H / 32;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -362,7 +370,7 @@ __global__ void gather_quant_kernel(const uint16_t* __restrict__ x, int H, int k
 // bf16 once.  8 bf16 per thread.
 __global__ void combine_kernel(const uint16_t* __restrict__ rows, const int32_t* __restrict__ inv,
                                const float* __restrict__ w, int T, int k, int H,
-                               uint16_t* __restrict__ out) {
+                               uint16_t* __restrict__ out, int* err) {
   const int nv = H / 8;
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (size_t)T * nv) return;
@@ -371,7 +379,12 @@ __global__ void combine_kernel(const uint16_t* __restrict__ rows, const int32_t*
   for (int j = 0; j < k; ++j) {
     const size_t slot = (size_t)t * k + j;
     const float wj = w ? __ldg(w + slot) : 1.f;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(rows + (size_t)__ldg(inv + slot) * H) + c);
+    const int32_t r = __ldg(inv + slot);
+    if (MXFP4_MOE_DEBUG && (r < 0 || r >= T * k)) {
+      DevErr{err}.set(MXFP4_MOE_ERR_DEVICE_BOUNDS, 0x112);
+      continue;
+    }
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(rows + (size_t)r * H) + c);
     a[0] += wj * bf16_lo(v.x); a[1] += wj * bf16_hi(v.x);
     a[2] += wj * bf16_lo(v.y); a[3] += wj * bf16_hi(v.y);
     a[4] += wj * bf16_lo(v.z); a[5] += wj * bf16_hi(v.z);
@@ -495,27 +508,27 @@ cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, 
 }
 
 cudaError_t launch_gather_rows(const uint16_t* src, int H, int k, const int32_t* perm, int A,
-                               uint16_t* dst, float* dot_w, cudaStream_t st) {
+                               uint16_t* dst, float* dot_w, int* err, cudaStream_t st) {
   const int threads = 256;
   const long long blocks = ((long long)A * 32 + threads - 1) / threads;
-  gather_rows_kernel<<<(unsigned)blocks, threads, 0, st>>>(src, H, k, perm, A, dst, dot_w);
+  gather_rows_kernel<<<(unsigned)blocks, threads, 0, st>>>(src, H, k, perm, A, dst, dot_w, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gather_quant(const uint16_t* x, int H, int k, const int32_t* perm, int A,
                                 uint8_t* hi, uint8_t* lo, uint8_t* sfb, int sfb_stride,
-                                cudaStream_t st) {
+                                int* err, cudaStream_t st) {
   const int threads = 256;
   const long long blocks = ((long long)A * 32 + threads - 1) / threads;
   gather_quant_kernel<<<(unsigned)blocks, threads, 0, st>>>(x, H, k, perm, A, hi, lo, sfb,
-                                                            sfb_stride);
+                                                            sfb_stride, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const uint16_t* rows, const int32_t* inv, const float* w, int T, int k,
-                           int H, uint16_t* out, cudaStream_t st) {
+                           int H, uint16_t* out, int* err, cudaStream_t st) {
   const size_t n = (size_t)T * (H / 8);
-  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rows, inv, w, T, k, H, out);
+  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rows, inv, w, T, k, H, out, err);
   return cudaGetLastError();
 }
 

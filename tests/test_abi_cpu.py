@@ -41,6 +41,20 @@ def test_library_exports_every_declared_symbol(L):
     assert set(syms) == set(L.SIGNATURES)
 
 
+def test_debug_build_exports_the_same_symbols_and_reports_itself(L):
+    """The debug build (device-side index checks) is the same boundary: every declared symbol,
+    and mxfp4_moe_build_flags tells the two builds apart (a host-only call)."""
+    from mxfp4_quantized_moe_b200 import build
+    dbg_path = build.build(debug=True)
+    rel = ctypes.CDLL(build.LIB)
+    dbg = ctypes.CDLL(dbg_path)
+    for s in declared_symbols():
+        assert hasattr(dbg, s), s
+    assert rel.mxfp4_moe_build_flags() == 0
+    assert dbg.mxfp4_moe_build_flags() == 1
+    assert L.lib.mxfp4_moe_build_flags() in (0, 1)
+
+
 def test_error_codes_match_header(L):
     src = open(HEADER).read()
     codes = dict(re.findall(r"#define (MXFP4_MOE_\w+) \(?(-?\d+)\)?", src))
