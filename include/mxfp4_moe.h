@@ -72,11 +72,22 @@ extern "C" {
 #define MXFP4_MOE_ERR_DEVICE_BOUNDS (-6)        /* a device-side index check failed        */
 
 /* Problem shape and GLU constants (GPT-OSS: glu_alpha = 1.702, glu_limit = 7).
- * Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", section "What this does" (the GptOssExperts expert loop and its activation). */
+ * Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", section "What this does" (the GptOssExperts expert loop and its activation).
+ * gate_up_format selects the operands of the forward's gate_up GEMM:
+ *   MXFP4_MOE_GATE_UP_BF16 (0, what a zero-initialised struct gives): the weights dequantized
+ *     to bf16 on the fly against the bf16 token rows;
+ *   MXFP4_MOE_GATE_UP_BLOCK_SCALED (1): the weights' E2M1 codes and UE8M0 scales as stored
+ *     against the token rows split into two E4M3 parts with a UE8M0 scale per 32 elements, on
+ *     the block-scaled tensor-core MMA ("Integrate finegrained kernels: SOTA performance and
+ *     per-module quantization", the commits on the activation format and input recipe).
+ * Any other value is INVALID_ARG.  The backward is the same for both. */
+#define MXFP4_MOE_GATE_UP_BF16 0
+#define MXFP4_MOE_GATE_UP_BLOCK_SCALED 1
 typedef struct {
   int32_t T, H, I, E, k;
   float glu_alpha;
   float glu_limit;
+  int32_t gate_up_format;
 } mxfp4_moe_dims;
 
 /* Frozen expert weights in the packed MXFP4 layout (read only, never modified).

@@ -33,7 +33,11 @@ _sz = ctypes.c_size_t
 class Dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("glu_alpha", ctypes.c_float),
-                ("glu_limit", ctypes.c_float)]
+                ("glu_limit", ctypes.c_float), ("gate_up_format", ctypes.c_int32)]
+
+
+GATE_UP_BF16 = 0
+GATE_UP_BLOCK_SCALED = 1
 
 
 class Weights(ctypes.Structure):

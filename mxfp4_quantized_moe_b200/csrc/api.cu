@@ -74,6 +74,9 @@ int check_dims(const mxfp4_moe_dims* d) {
   if (d->E < 1 || d->E > 256 || d->k < 1 || d->k > d->E) return MXFP4_MOE_ERR_INVALID_ARG;
   if ((long long)d->T * d->k >= (1ll << 31)) return MXFP4_MOE_ERR_INVALID_ARG;
   if (!(d->glu_limit > 0.f) || !(d->glu_alpha == d->glu_alpha)) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (d->gate_up_format != MXFP4_MOE_GATE_UP_BF16 &&
+      d->gate_up_format != MXFP4_MOE_GATE_UP_BLOCK_SCALED)
+    return MXFP4_MOE_ERR_INVALID_ARG;
   // the grouped GEMM keeps a tile's scales for the whole contraction in shared memory
   if (moe::grouped_gemm_smem_bytes(d->H > 2 * d->I ? d->H : 2 * d->I, 0) > 232448 ||
       moe::grouped_gemm_smem_bytes(d->H, sfb_stride(d->H)) > 232448)
@@ -257,22 +260,30 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
 
   MOE_LAUNCH("router_topk", moe::launch_router_topk(logits, T, E, k, idx, wr, blk_hist, topk_idx, topk_w, st));
   MOE_LAUNCH("build_perm", moe::launch_build_perm(idx, wr, T, E, k, blk_hist, off, perm, inv, w_row, err, st));
-  // Xp in expert-sorted order as two E4M3 parts (hi | lo in the dH region, free until the
-  // backward) with UE8M0 block scales
+  const bool bs = d->gate_up_format == MXFP4_MOE_GATE_UP_BLOCK_SCALED;
+  // Xp in expert-sorted order: bf16 rows (in `rows`, which the down GEMM overwrites with y), or
+  // as two E4M3 parts (hi | lo in the dH region, free until the backward) with UE8M0 scales
   uint8_t* xhi = at<uint8_t>(ws, L.dh);
   uint8_t* xlo = xhi + (size_t)A * H;
   uint8_t* sfb = at<uint8_t>(ws, L.sfb);
-  MOE_LAUNCH("gather_x_mx", moe::launch_gather_quant(x, H, k, perm, A, xhi, xlo, sfb, sfb_stride(H), err, st));
+  if (bs)
+    MOE_LAUNCH("gather_x_mx", moe::launch_gather_quant(x, H, k, perm, A, xhi, xlo, sfb, sfb_stride(H), err, st));
+  else
+    MOE_LAUNCH("gather_x", moe::launch_gather_rows(x, H, k, perm, A, rows, nullptr, err, st));
 
   moe::GemmArgs g{};
   g.off = off; g.E = E; g.A = A; g.err = err;
   g.alpha = d->glu_alpha; g.limit = d->glu_limit; g.mask_limit = bf16_mask_limit(d->glu_limit);
   // gate_up: h = Xp W_gu^T + b_gu; act = GLU(h) and the GLU derivative factors are saved
-  // (block-scaled: E2M1 weights against the E4M3 parts, fp32 accumulation)
+  // (block-scaled: E2M1 weights against the E4M3 parts; both forms accumulate in fp32)
   g.scales = w->gu_scales; g.K = H; g.N = 2 * I; g.bias = w->gu_bias; g.out0 = dgu; g.out1 = act;
-  g.tok_lo = xlo; g.sfb = sfb; g.sfb_stride = sfb_stride(H);
-  MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, xhi, w->gu_blocks, g, sms, st));
-  g.tok_lo = nullptr; g.sfb = nullptr; g.sfb_stride = 0;
+  if (bs) {
+    g.tok_lo = xlo; g.sfb = sfb; g.sfb_stride = sfb_stride(H);
+    MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, xhi, w->gu_blocks, g, sms, st));
+    g.tok_lo = nullptr; g.sfb = nullptr; g.sfb_stride = 0;
+  } else {
+    MOE_LAUNCH("gemm_gate_up_glu", moe::launch_grouped_gemm(moe::kEpiGateUp, false, rows, w->gu_blocks, g, sms, st));
+  }
   // down: y = act W_d^T + b_d per sorted row (kept for the backward's routing-weight gradient)
   g.scales = w->dn_scales; g.K = I; g.N = H; g.bias = w->dn_bias; g.out0 = rows; g.out1 = nullptr;
   MOE_LAUNCH("gemm_down", moe::launch_grouped_gemm(moe::kEpiDown, false, act, w->dn_blocks, g, sms, st));

@@ -22,8 +22,13 @@
 //   warps 12-15 epilogue: TMEM -> registers -> fused bias / GLU / routing / scatter
 // The token and weight rings are separate so that the converters can run ahead of the MMA
 // by the depth of the TMEM A ring without pinning token stages.
-// TMEM (512 columns): two fp32 accumulators of kBN columns (double buffered across tiles)
-// and a 4-stage ring of A operands (32 columns = 64 bf16 of K each).
+// TMEM (512 columns): one fp32 accumulator of kBN = 256 columns and a 4-stage ring of A
+// operands (32 columns = 64 bf16 of K each).  The epilogue releases the accumulator as soon as
+// it holds the tile in registers (rounded to bf16, two columns per word), so the next tile's
+// MMAs overlap the processing and stores of this one; dact, which multiplies the fp32 values,
+// releases it after its last chunk.  An MMA instruction costs time in proportion to N from
+// N = 128 up (half a cycle per column per K=16 step), and a k-step's fixed costs (barrier
+// round trips, conversion) do not grow with N, so the widest tile amortizes them best.
 //
 // Which weights: the forward GEMMs read the stored rows (scales per row and 32-element
 // block of K).  The backward GEMMs contract over the stored rows' output axis, so they
@@ -50,13 +55,20 @@ namespace {
 constexpr int kStages = 4;        // even: a stage always belongs to the same converter parity
 // Publish and issue each k-step on its own (true) or the two k-steps of a pair together (false).
 constexpr bool kStageIssue = true;
-constexpr int kWStages = 8;       // packed-weight ring depth (even, same reason)
+// packed-weight ring depth (even, same reason): 8 stages, 4 in the block-scaled form, whose
+// per-tile token scales take the shared memory the other four would
+constexpr int kWStagesMax = 8;
+template <bool BS>
+__host__ __device__ constexpr int wstages() { return BS ? 4 : kWStagesMax; }
 constexpr int kThreads = 512;
 constexpr int kConvWarps = 8;
-constexpr int kTokBytes = kBN * kBK * 2;      // 24 KB
+constexpr int kTokBytes = kBN * kBK * 2;      // 32 KB
 constexpr int kWBytes = kBM * (kBK / 2);      // 4 KB of packed nibbles
 constexpr int kAccCols = kBN;                 // fp32 accumulator columns per buffer
-constexpr int kACol0 = 2 * kAccCols;          // first TMEM column of the A ring
+// One accumulator of kBN = 256 columns: the epilogue releases it as soon as it holds the tile
+// in registers (two accumulators of 256 columns would leave no room for the A ring).
+constexpr int kAccBufs = 1;
+constexpr int kACol0 = kAccBufs * kAccCols;   // first TMEM column of the A ring
 constexpr int kTmemCols = 512;
 // Registers per thread by warpgroup after setmaxnreg: control (producers, MMA, warpgroup 0),
 // converters (warpgroups 1-2), epilogue (warpgroup 3).  setmaxnreg.inc draws only on what the
@@ -81,15 +93,16 @@ constexpr int kSfbCol0 = kSfaCol0 + kStages * 4;
 static_assert(kSfbCol0 + kStages * 8 <= kTmemCols, "TMEM budget (block-scaled)");
 static_assert(kSfbCols <= 8, "scale-factor columns of the token tile");
 static_assert(kBN % 32 == 0 && kBN <= 256, "token tile");
-static_assert(kWStages % 2 == 0 && kStages % 2 == 0, "ring depths must be even");
+static_assert(wstages<false>() % 2 == 0 && wstages<true>() % 2 == 0 && kStages % 2 == 0,
+              "ring depths must be even");
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 struct __align__(8) Barriers {
   uint64_t full[kStages];   // token bytes landed + 4 converter warps stored the A operand
   uint64_t empty[kStages];  // MMA commit: token stage and A stage free again
-  uint64_t w_full[kWStages];
-  uint64_t w_empty[kWStages];
+  uint64_t w_full[kWStagesMax];
+  uint64_t w_empty[kWStagesMax];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t sc_full[2];
@@ -98,17 +111,19 @@ struct __align__(8) Barriers {
 };
 static_assert(sizeof(Barriers) <= 512, "barrier block");
 
-struct SmemLayout {
+template <bool BS>
+struct SmemLayoutT {
   // offsets from the 1024-aligned dynamic smem base
   static constexpr int tok = 0;                                  // 1024-aligned (128B swizzle)
   static constexpr int w = tok + kStages * kTokBytes;            // 256-aligned (32B swizzle)
-  static constexpr int bars = w + kWStages * kWBytes;
+  static constexpr int bars = w + wstages<BS>() * kWBytes;
   static constexpr int misc = bars + 512;                        // tmem slot, abort flag
   static constexpr int cw = misc + 64;                           // 8 warps x 4 x 32 scale words
   static constexpr int tables = cw + kConvWarps * 4 * 32 * 4;    // off[257], tile_start[257]
   static constexpr int sc = ((tables + 2 * 257 * 4) + 127) / 128 * 128;  // 2 scale buffers
 };
-static_assert(SmemLayout::w % 1024 == 0, "weight ring alignment");
+static_assert(SmemLayoutT<false>::w % 1024 == 0 && SmemLayoutT<true>::w % 1024 == 0,
+              "weight ring alignment");
 
 template <uint32_t N>
 MOE_DEV void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
@@ -120,7 +135,8 @@ struct Tile {
 };
 
 // An expert's m rows are split into equal token tiles of at most kBN rows (a multiple of 16),
-// so that no tile is a small remainder: the MMA costs nearly the same at N = 64 as at N = 192.
+// so that no tile is a small remainder: a k-step's fixed costs are the same for a tile of 32
+// rows as for one of 256.
 MOE_DEV int token_tile_rows(int m) {
   const int n = (m + kBN - 1) / kBN;
   const int rows = (m + n - 1) / n;
@@ -166,6 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmap_lo,
                         const __grid_constant__ CUtensorMap tmap_w, const GemmArgs p) {
   static_assert(!BS || (EPI == kEpiGateUp && !COLT), "block-scaled form: gate_up only");
+  using SmemLayout = SmemLayoutT<BS>;
+  constexpr int kWStages = wstages<BS>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -331,8 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
           Tile tl;
           decode_tile(t, s_tstart, s_off, E, nfb, tl);
-          const int acc = lt & 1;
-          if (!mbar_wait(smem_u32(&bar->acc_empty[acc]), ((lt >> 1) & 1) ^ 1, err, 0x300, s_abort)) break;
+          const int acc = lt % kAccBufs;
+          if (!mbar_wait(smem_u32(&bar->acc_empty[acc]), ((lt / kAccBufs) & 1) ^ 1, err, 0x300, s_abort)) break;
           tc_fence_after();
           const uint32_t idesc = idesc_bf16_m128((tl.n_valid + 15) & ~15);
           const uint32_t d_tmem = tmem + acc * kAccCols;
@@ -683,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
       Tile tl;
       decode_tile(t, s_tstart, s_off, E, nfb, tl);
-      const int acc = lt & 1;
+      const int acc = lt % kAccBufs;
       const int f = tl.feat0 + 32 * q + lane;  // output feature of this thread
       const bool active = tl.feat0 + 32 * q < N;
       // dact: the saved GLU factors of the tile's first 32 rows are requested before the
@@ -694,128 +712,167 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j)
           dnext[j] = __ldg(p.dgu + (size_t)min(tl.row0 + j, p.A - 1) * N + f);
       }
-      if (!mbar_wait_sleep(smem_u32(&bar->acc_full[acc]), (lt >> 1) & 1, err, 0x500, s_abort, 256)) break;
+      if (!mbar_wait_sleep(smem_u32(&bar->acc_full[acc]), (lt / kAccBufs) & 1, err, 0x500, s_abort, 256)) break;
       tc_fence_after();
       float bias_f = 0.f;
       if ((EPI == kEpiGateUp || EPI == kEpiDown) && active)
         bias_f = bf16_to_f(p.bias[(size_t)tl.e * N + f]);
-      for (int c0 = 0; c0 < tl.n_valid; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + acc * kAccCols + c0, r);
-        tmem_wait_ld();
-        if (!active) continue;
-        const int ncol = min(32, tl.n_valid - c0);
-        const int rbase = tl.row0 + c0;
-        const bool odd = (lane & 1) != 0;
-        if (EPI == kEpiGateUp) {
-          // Columns j (even lane) and j+1 (odd lane) of each pair: the lanes of an
-          // interleaved (gate, up) feature pair swap one value so that each holds (g, u) of
-          // its own column.  Stored per (row, j): act = (u'+1) g' sigmoid(a g') and, for the
-          // backward, the GLU derivative factors d act/d g and d act/d u as one bf16x2 word
-          // (clamp masks decided on h rounded to bf16, as the eager bf16 model holds it).
-          const int I = N >> 1;
-          const int jf = f >> 1;
-          uint32_t dw16[16];
-          float av[16];
-          // two columns per step with the paired fp32 instructions (same operations and
-          // rounding as one column at a time)
-          const uint64_t kBias = f2(bias_f, bias_f), kOne = f2(1.f, 1.f);
-          const uint64_t kHalfAlpha = f2(0.5f * p.alpha, 0.5f * p.alpha);
-          const uint64_t kHalf = f2(0.5f, 0.5f), kAlpha = f2(p.alpha, p.alpha);
-          const uint64_t kMinusOne = f2(-1.f, -1.f);
+      const uint32_t acc_tmem = tmem + ((uint32_t)(32 * q) << 16) + acc * kAccCols;
+      const bool odd = (lane & 1) != 0;
+      if (EPI != kEpiDact) {
+        // Early release: the tile's accumulator, bias added and rounded to bf16 (two columns
+        // per word), moves into registers first; the MMA may start the next tile as soon as
+        // every epilogue warp holds its rows, while the values are processed and stored.
+        // down and dx store exactly these bf16 values; gate_up evaluates the GLU on them
+        // (h rounded to bf16, as the eager bf16 model holds it).
+        uint32_t pk[kBN / 32][16];
 #pragma unroll
-          for (int jj = 0; jj < 16; jj += 2) {
-            const uint64_t va = f2add(f2(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 2])), kBias);
-            const uint64_t vb = f2add(f2(__uint_as_float(r[2 * jj + 1]), __uint_as_float(r[2 * jj + 3])), kBias);
-            const float v0a = f2lo(va), v0b = f2hi(va), v1a = f2lo(vb), v1b = f2hi(vb);
-            const float ra = __shfl_xor_sync(kFull, odd ? v0a : v1a, 1);
-            const float rb = __shfl_xor_sync(kFull, odd ? v0b : v1b, 1);
-            const float ga = odd ? ra : v0a, ua = odd ? v1a : ra;
-            const float gb = odd ? rb : v0b, ub = odd ? v1b : rb;
-            const uint64_t gc = f2(fminf(ga, p.limit), fminf(gb, p.limit));
-            const uint64_t uc = f2(fminf(fmaxf(ua, -p.limit), p.limit), fminf(fmaxf(ub, -p.limit), p.limit));
-            // sigmoid(a g') = (1 + tanh(a g' / 2)) / 2
-            const uint64_t z = f2mul(kHalfAlpha, gc);
-            float ta, tb;
-            asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(f2lo(z)));
-            asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(f2hi(z)));
-            const uint64_t sg = f2fma(kHalf, f2(ta, tb), kHalf);
-            const uint64_t t1 = f2mul(gc, sg);
-            const uint64_t up1 = f2add(uc, kOne);
-            const uint64_t act = f2mul(up1, t1);
-            av[jj] = f2lo(act);
-            av[jj + 1] = f2hi(act);
-            // d act / d g' = (u'+1) (s + a t1 (1 - s)); d act / d u' = t1
-            const uint64_t om = f2fma(sg, kMinusOne, kOne);
-            const uint64_t dg = f2mul(up1, f2fma(f2mul(kAlpha, t1), om, sg));
-            // bf16(g) <= limit  <=>  g <= mask_limit (and likewise for |bf16(u)|)
-            const float dga = (ga <= p.mask_limit) ? f2lo(dg) : 0.f;
-            const float dgb = (gb <= p.mask_limit) ? f2hi(dg) : 0.f;
-            const float dua = (fabsf(ua) <= p.mask_limit) ? f2lo(t1) : 0.f;
-            const float dub = (fabsf(ub) <= p.mask_limit) ? f2hi(t1) : 0.f;
-            dw16[jj] = pack_bf16x2(dga, dua);
-            dw16[jj + 1] = pack_bf16x2(dgb, dub);
+        for (int c = 0; c < kBN / 32; ++c) {
+          if (32 * c < tl.n_valid) {
+            uint32_t r[32];
+            tmem_ld32(acc_tmem + 32 * c, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              pk[c][jj] = pack_bf16x2(__uint_as_float(r[2 * jj]) + bias_f,
+                                      __uint_as_float(r[2 * jj + 1]) + bias_f);
           }
-          uint32_t* dgu_out = reinterpret_cast<uint32_t*>(p.out0);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar->acc_empty[acc]));
+        if (active) {
+          // the work on one chunk of 32 columns (the tile's rows rbase .. rbase + ncol - 1)
+          auto chunk = [&](const uint32_t (&cur)[16], int ncol, int rbase) {
+            if (EPI == kEpiGateUp) {
+              // Columns j (even lane) and j+1 (odd lane) of each pair: the lanes of an
+              // interleaved (gate, up) feature pair swap one value so that each holds (g, u)
+              // of its own column.  Stored per (row, j): act = (u'+1) g' sigmoid(a g') and,
+              // for the backward, the GLU derivative factors d act/d g and d act/d u as one
+              // bf16x2 word.
+              const int I = N >> 1;
+              const int jf = f >> 1;
+              uint32_t dw16[16];
+              float av[16];
+              // two columns per step with the paired fp32 instructions (same operations and
+              // rounding as one column at a time)
+              const uint64_t kOne = f2(1.f, 1.f);
+              const uint64_t kHalfAlpha = f2(0.5f * p.alpha, 0.5f * p.alpha);
+              const uint64_t kHalf = f2(0.5f, 0.5f), kAlpha = f2(p.alpha, p.alpha);
+              const uint64_t kMinusOne = f2(-1.f, -1.f);
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int col = 2 * jj + (odd ? 1 : 0);
-            if (col < ncol) {
-              const size_t o = (size_t)(rbase + col) * I + jf;
-              dgu_out[o] = dw16[jj];
-              p.out1[o] = f_to_bf16(av[jj]);
-            }
-          }
-        } else {
-          if (EPI == kEpiDown || EPI == kEpiDx) {
-            // Feature pairs (f, f+1) live in lanes (2m, 2m+1): after one swap the even lane
-            // holds both features of column j, the odd lane both of column j+1.  Rows are
-            // stored in expert-sorted order (down: y = act W_d^T + b_d, not yet weighted; the
-            // combine applies the routing weights).
-            uint32_t ow[16];
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              float v0 = __uint_as_float(r[2 * jj]);
-              float v1 = __uint_as_float(r[2 * jj + 1]);
-              if (EPI == kEpiDown) {
-                v0 += bias_f;
-                v1 += bias_f;
+              for (int jj = 0; jj < 16; jj += 2) {
+                const uint32_t wa = cur[jj], wb = cur[jj + 1];  // columns 2jj, 2jj+1 | +2, +3
+                const float v0a = bf16_lo(wa), v0b = bf16_lo(wb), v1a = bf16_hi(wa), v1b = bf16_hi(wb);
+                const float ra = __shfl_xor_sync(kFull, odd ? v0a : v1a, 1);
+                const float rb = __shfl_xor_sync(kFull, odd ? v0b : v1b, 1);
+                const float ga = odd ? ra : v0a, ua = odd ? v1a : ra;
+                const float gb = odd ? rb : v0b, ub = odd ? v1b : rb;
+                const uint64_t gc = f2(fminf(ga, p.limit), fminf(gb, p.limit));
+                const uint64_t uc = f2(fminf(fmaxf(ua, -p.limit), p.limit), fminf(fmaxf(ub, -p.limit), p.limit));
+                // sigmoid(a g') = (1 + tanh(a g' / 2)) / 2
+                const uint64_t z = f2mul(kHalfAlpha, gc);
+                float ta, tb;
+                asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(f2lo(z)));
+                asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(f2hi(z)));
+                const uint64_t sg = f2fma(kHalf, f2(ta, tb), kHalf);
+                const uint64_t t1 = f2mul(gc, sg);
+                const uint64_t up1 = f2add(uc, kOne);
+                const uint64_t act = f2mul(up1, t1);
+                av[jj] = f2lo(act);
+                av[jj + 1] = f2hi(act);
+                // d act / d g' = (u'+1) (s + a t1 (1 - s)); d act / d u' = t1
+                const uint64_t om = f2fma(sg, kMinusOne, kOne);
+                const uint64_t dg = f2mul(up1, f2fma(f2mul(kAlpha, t1), om, sg));
+                // bf16(g) <= limit  <=>  g <= mask_limit (and likewise for |bf16(u)|)
+                const float dga = (ga <= p.mask_limit) ? f2lo(dg) : 0.f;
+                const float dgb = (gb <= p.mask_limit) ? f2hi(dg) : 0.f;
+                const float dua = (fabsf(ua) <= p.mask_limit) ? f2lo(t1) : 0.f;
+                const float dub = (fabsf(ub) <= p.mask_limit) ? f2hi(t1) : 0.f;
+                dw16[jj] = pack_bf16x2(dga, dua);
+                dw16[jj + 1] = pack_bf16x2(dgb, dub);
               }
-              const float recv = __shfl_xor_sync(kFull, odd ? v0 : v1, 1);
-              ow[jj] = odd ? pack_bf16x2(recv, v1) : pack_bf16x2(v0, recv);
+              uint32_t* dgu_out = reinterpret_cast<uint32_t*>(p.out0);
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) {
+                const int col = 2 * jj + (odd ? 1 : 0);
+                if (col < ncol) {
+                  const size_t o = (size_t)(rbase + col) * I + jf;
+                  dgu_out[o] = dw16[jj];
+                  p.out1[o] = f_to_bf16(av[jj]);
+                }
+              }
+            } else {
+              // Feature pairs (f, f+1) live in lanes (2m, 2m+1), each lane holding its feature
+              // for the columns (2jj, 2jj+1): after one swap of whole words the even lane
+              // holds both features of column 2jj, the odd lane both of column 2jj+1.  Rows
+              // are stored in expert-sorted order (down: y = act W_d^T + b_d, not yet
+              // weighted; the combine applies the routing weights).
+              uint32_t* orow = reinterpret_cast<uint32_t*>(p.out0);
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) {
+                const uint32_t w = cur[jj];
+                const uint32_t wp = __shfl_xor_sync(kFull, w, 1);
+                const uint32_t ow = odd ? prmt(wp, w, 0x7632u) : prmt(w, wp, 0x5410u);
+                const int col = 2 * jj + (odd ? 1 : 0);
+                if (col < ncol) orow[((size_t)(rbase + col) * N + (f & ~1)) >> 1] = ow;
+              }
             }
-            uint32_t* orow = reinterpret_cast<uint32_t*>(p.out0);
+          };
+          if (EPI == kEpiGateUp) {
+            // one chunk per pass, always from pk[0]: the chunks move down one slot per pass,
+            // so the GLU is emitted once (eight unrolled copies would crowd the instruction
+            // cache that the converters and the MMA issuer run from)
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+              if (32 * c >= tl.n_valid) break;
+              chunk(pk[0], min(32, tl.n_valid - 32 * c), tl.row0 + 32 * c);
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              const int col = 2 * jj + (odd ? 1 : 0);
-              if (col < ncol) orow[((size_t)(rbase + col) * N + (f & ~1)) >> 1] = ow[jj];
+              for (int cc = 0; cc + 1 < kBN / 32; ++cc)
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) pk[cc][jj] = pk[cc + 1][jj];
             }
-          } else {  // kEpiDact
-            // dZ = dY W_d for this row; dact = w dZ; dH = (dact * dact/dg, dact * dact/du)
-            // from the factors the forward saved.
-            const int I = N;
-            uint32_t* dh = reinterpret_cast<uint32_t*>(p.out0);
-            const float my_w = (lane < ncol) ? p.w_row[rbase + lane] : 0.f;
-            uint32_t dcur[32];
+          } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dcur[j] = dnext[j];
-            if (c0 + 32 < tl.n_valid) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                dnext[j] = __ldg(p.dgu + (size_t)min(rbase + 32 + j, p.A - 1) * I + f);
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float dact = __shfl_sync(kFull, my_w, j) * __uint_as_float(r[j]);
-              const uint32_t dh2 = pack_bf16x2(dact * bf16_lo(dcur[j]), dact * bf16_hi(dcur[j]));
-              if (j < ncol) dh[(size_t)(rbase + j) * I + f] = dh2;
+            for (int c = 0; c < kBN / 32; ++c) {
+              if (32 * c >= tl.n_valid) break;
+              chunk(pk[c], min(32, tl.n_valid - 32 * c), tl.row0 + 32 * c);
             }
           }
         }
+      } else {
+        // dact keeps the fp32 accumulator through its multiply: chunk by chunk, then release
+        for (int c0 = 0; c0 < tl.n_valid; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(acc_tmem + c0, r);
+          tmem_wait_ld();
+          if (!active) continue;
+          const int ncol = min(32, tl.n_valid - c0);
+          const int rbase = tl.row0 + c0;
+          // dZ = dY W_d for this row; dact = w dZ; dH = (dact * dact/dg, dact * dact/du)
+          // from the factors the forward saved.
+          const int I = N;
+          uint32_t* dh = reinterpret_cast<uint32_t*>(p.out0);
+          const float my_w = (lane < ncol) ? p.w_row[rbase + lane] : 0.f;
+          uint32_t dcur[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dcur[j] = dnext[j];
+          if (c0 + 32 < tl.n_valid) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              dnext[j] = __ldg(p.dgu + (size_t)min(rbase + 32 + j, p.A - 1) * I + f);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float dact = __shfl_sync(kFull, my_w, j) * __uint_as_float(r[j]);
+            const uint32_t dh2 = pack_bf16x2(dact * bf16_lo(dcur[j]), dact * bf16_hi(dcur[j]));
+            if (j < ncol) dh[(size_t)(rbase + j) * I + f] = dh2;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar->acc_empty[acc]));
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar->acc_empty[acc]));
     }
     __syncwarp();
     __syncthreads();
@@ -879,7 +936,8 @@ bool encode_2d(EncodeTiledFn enc, CUtensorMap* m, CUtensorMapDataType type, cons
 }  // namespace
 
 size_t grouped_gemm_smem_bytes(int K, int sfb_stride) {
-  return 1024 + SmemLayout::sc + 2 * ((size_t)(4 * K) + (size_t)kBN * sfb_stride);
+  return 1024 + (sfb_stride ? SmemLayoutT<true>::sc : SmemLayoutT<false>::sc) +
+         2 * ((size_t)(4 * K) + (size_t)kBN * sfb_stride);
 }
 
 cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const void* tokens,

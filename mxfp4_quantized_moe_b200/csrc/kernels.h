@@ -16,7 +16,7 @@ namespace moe {
 // Tile shape of the grouped GEMMs: 128 weight rows (output features) in TMEM as the
 // MMA's A operand, BN routed tokens per tile in shared memory as the B operand.
 constexpr int kBM = 128;
-constexpr int kBN = 192;
+constexpr int kBN = 256;
 constexpr int kBK = 64;
 
 enum Epilogue : int { kEpiGateUp = 0, kEpiDown = 1, kEpiDact = 2, kEpiDx = 3 };

@@ -6,8 +6,8 @@
   set, E*2I rows of H elements: 0.5 B of codes + 1/32 B of scale read and 2 B of bf16 written
   per element;
 * the memory-bound kernels of one gpt-oss-20b layer step at T=8192, from the library's
-  per-kernel event timing: the forward gather with the MX split (`gather_x_mx`: A rows of H
-  bf16 read, the E4M3 hi and lo parts and one scale byte per 32 written), the combines
+  per-kernel event timing: the forward gather (`gather_x`: A rows of H bf16 read and
+  written), the combines
   (`combine_y`, `combine_dx`: A rows read, T rows written) and the dY gather with the
   routing-weight dot (`gather_dy_dw`: A rows of dY and of y read, A rows written).
 
@@ -84,8 +84,7 @@ def main():
         moe.backward_input(shape, w, wt, dy, ws)
     kt = moe.profile_end()
     A, T, H = wl.T * wl.k, wl.T, wl.H
-    sfb_stride = (2 * (-(-H // 64)) + 31) // 32 * 32
-    stages = (("gather_x_mx", A * H * 2.0 + A * H * 2.0 + A * sfb_stride),
+    stages = (("gather_x", A * H * 2.0 * 2),
               ("combine_y", (A + T) * H * 2.0),
               ("gather_dy_dw", A * H * 2.0 * 3 + A * 4.0),
               ("combine_dx", (A + T) * H * 2.0))

@@ -25,9 +25,13 @@ class MoeShape:
     k: int
     glu_alpha: float = 1.702
     glu_limit: float = 7.0
+    # forward gate_up operands: 0 = bf16 (weights dequantized on the fly), 1 = block-scaled
+    # (E2M1 weights as stored against E4M3 hi / lo token parts with UE8M0 block scales)
+    gate_up_format: int = 0
 
     def dims(self) -> Dims:
-        return Dims(self.T, self.H, self.I, self.E, self.k, self.glu_alpha, self.glu_limit)
+        return Dims(self.T, self.H, self.I, self.E, self.k, self.glu_alpha, self.glu_limit,
+                    self.gate_up_format)
 
 
 def _ptr(t: torch.Tensor | None):

@@ -55,6 +55,13 @@ def test_debug_build_exports_the_same_symbols_and_reports_itself(L):
     assert L.lib.mxfp4_moe_build_flags() in (0, 1)
 
 
+def test_unknown_gate_up_format_is_rejected(L):
+    n = ctypes.c_size_t()
+    for fmt, want in ((0, L.OK), (1, L.OK), (2, L.ERR_INVALID_ARG), (-1, L.ERR_INVALID_ARG)):
+        d = L.Dims(64, 256, 256, 8, 2, 1.702, 7.0, fmt)
+        assert L.lib.mxfp4_moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == want, fmt
+
+
 def test_error_codes_match_header(L):
     src = open(HEADER).read()
     codes = dict(re.findall(r"#define (MXFP4_MOE_\w+) \(?(-?\d+)\)?", src))

@@ -74,9 +74,9 @@ def assert_d_logits_close(got, ref, w, d_w, name="d_logits", require_resolved=Fa
         assert_close(got[resolved[:, 0]], ref[resolved[:, 0]], name)
 
 
-def run_block(moe, T, H, I, E, k, seed, tokens=None, **kw):
+def run_block(moe, T, H, I, E, k, seed, tokens=None, gate_up_format=0, **kw):
     inp = inputs.make_layer(T, H, I, E, k, seed, **kw)
-    shape = moe.MoeShape(T, H, I, E, k)
+    shape = moe.MoeShape(T, H, I, E, k, gate_up_format=gate_up_format)
     w = moe.weights_to(inp, "cuda")
     x, lg, dy = inp["x"].cuda(), inp["logits"].cuda(), inp["dy"].cuda()
     ws = moe.alloc_workspace(shape)
@@ -208,6 +208,18 @@ def test_edge_cases(moe, T, H, I, E, k, seed, kw):
     check_all(got, ref)
 
 
+@pytest.mark.parametrize("T,H,I,E,k,seed,tokens", [
+    (64, 256, 256, 8, 2, 0, None),        # the tiny workload, every token
+    (37, 96, 160, 5, 3, 4, None),         # K tails, ragged tiles
+    (300, 2880, 2880, 32, 4, 13, None),   # gpt-oss-20b widths, every token
+])
+def test_block_scaled_gate_up_parity(moe, T, H, I, E, k, seed, tokens):
+    """The forward with the block-scaled gate_up (E2M1 weights as stored against the E4M3
+    hi / lo split of the token rows): the whole block against the oracle, like the bf16 form."""
+    got, ref = run_block(moe, T, H, I, E, k, seed, tokens=tokens, gate_up_format=1)
+    check_all(got, ref)
+
+
 @pytest.mark.parametrize("T", [1, 64, 256])
 def test_small_token_gpt_oss_20b_every_token(moe, T):
     """The small-token (decode-sized) batches of the gpt-oss-20b layer (H=I=2880, E=32, k=4),
@@ -224,7 +236,7 @@ def test_expert_gradient_is_not_silent(moe):
     check_all(got, ref)
 
 
-def tile_boundary_tokens(logits, k, cap, seed, tile_rows=192):
+def tile_boundary_tokens(logits, k, cap, seed, tile_rows=256):
     """Tokens whose assignments sit on the first or last row of a grouped-GEMM token tile.
 
     The GEMMs cut each expert's m expert-sorted rows into ceil(m / tile_rows) equal tiles of
@@ -379,7 +391,7 @@ def test_activation_split_matches_the_mx_definition(moe):
     x[5, :32] = 0.0         # an all-zero block
     x[7, 32:64] *= 2 ** 40  # a large block
     x[9, 64:96] *= 2 ** -40  # a small block, elements far below the rest of the row
-    shape = moe.MoeShape(T, H, I, E, k)
+    shape = moe.MoeShape(T, H, I, E, k, gate_up_format=1)
     w = moe.weights_to(inp, "cuda")
     ws = moe.alloc_workspace(shape)
     moe.forward(shape, w, x.cuda(), inp["logits"].cuda(), ws)

@@ -26,7 +26,7 @@ import torch
 from mxfp4_quantized_moe_b200 import inputs, stack
 
 import oracle_pool
-from test_gpu_parity import assert_close, assert_d_logits_close
+from test_gpu_parity import _ws_offsets, assert_close, assert_d_logits_close
 
 pytestmark = pytest.mark.gpu
 
@@ -46,8 +46,15 @@ def _run_blockwise(wl, seed, sel, workers=1):
     def tap_f(l, d):
         fw[l] = {k: d[k][selc].cpu() for k in ("x", "logits", "y")}
 
+    o = _ws_offsets(wl.T, wl.E, wl.k)
+    nA = wl.T * wl.k
+
     def tap_b(l, d):
         bw[l] = {k: d[k][selc].cpu() for k in ("g", "dx", "d_logits", "d_w")}
+        # the routing the block's backward used (its recomputed forward's, in the workspace)
+        ws = st.ws
+        bw[l]["idx"] = ws[o["idx"]:o["idx"] + 4 * nA].view(torch.int32).view(wl.T, wl.k)[selc].cpu()
+        bw[l]["w"] = ws[o["w"]:o["w"] + 4 * nA].view(torch.float32).view(wl.T, wl.k)[selc].cpu()
 
     st = stack.MoeStack(shape, blocks)
     out, saved = st.forward(x, tap=tap_f)
@@ -77,12 +84,14 @@ def _run_blockwise(wl, seed, sel, workers=1):
         gdl = _np(bw[l]["d_logits"])
         # d_logits against the oracle, with the per-token floor of the bf16 rounding of y
         assert_d_logits_close(gdl, d_logits, w, d_w, f"d_logits[{l}]", y_abs=y_abs)
-        # the softmax Jacobian itself, applied in fp64 to the GPU's own d_w: fp32-exact
-        idx = np.argsort(-fw[l]["logits"].double().numpy(), axis=1, kind="stable")[:, :wl.k]
-        sel = w * (gdw - (w * gdw).sum(axis=1, keepdims=True))
+        # the softmax Jacobian itself, applied in fp64 to the GPU's own routing (its top-k
+        # and weights, which a near tie in the logits can set apart from the oracle's) and d_w
+        gi = bw[l]["idx"].numpy().astype(np.int64)
+        gw = bw[l]["w"].double().numpy()
+        sel = gw * (gdw - (gw * gdw).sum(axis=1, keepdims=True))
         jac = np.zeros_like(gdl)
-        np.put_along_axis(jac, idx, sel, axis=1)
-        assert_d_logits_close(gdl, jac, w, gdw, f"d_logits[{l}] from the GPU's d_w")
+        np.put_along_axis(jac, gi, sel, axis=1)
+        assert_d_logits_close(gdl, jac, gw, gdw, f"d_logits[{l}] from the GPU's d_w")
 
 
 def test_small_stack_blockwise_all_tokens():
