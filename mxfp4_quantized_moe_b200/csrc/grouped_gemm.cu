@@ -53,8 +53,6 @@ namespace {
 // MMA-facing ring: stage s holds the token tile (shared memory) and the bf16 A operand
 // (TMEM) of one k-step; the MMA waits once and commits once per k-step.
 constexpr int kStages = 4;        // even: a stage always belongs to the same converter parity
-// Publish and issue each k-step on its own (true) or the two k-steps of a pair together (false).
-constexpr bool kStageIssue = true;
 // packed-weight ring depth (even, same reason): 8 stages, 4 in the block-scaled form, whose
 // per-tile token scales take the shared memory the other four would
 constexpr int kWStagesMax = 8;
@@ -354,101 +352,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t idesc = idesc_bf16_m128((tl.n_valid + 15) & ~15);
           const uint32_t d_tmem = tmem + acc * kAccCols;
-          if (kStageIssue) {
-            // one k-step per round: wait for its stage, issue its MMAs, release it on completion
-            const int npad = (tl.n_valid + 15) & ~15;
-            for (int ks = 0; ks < nk; ++ks) {
-              if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t tbase = tok_base + s * kTokBytes;
-              if (BS) {
-                const uint64_t bhi = smem_desc_kmajor_sw64(tbase);
-                const uint64_t blo = smem_desc_kmajor_sw64(tbase + kTokBytes / 2);
-                const uint32_t a_tmem = tmem + kACol0 + s * kAColsBS;
-                const uint32_t sfa = tmem + kSfaCol0 + s * 4, sfb = tmem + kSfbCol0 + s * 8;
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                  const uint32_t id = idesc_mxf4a_m128(npad, (uint32_t)kk);
-                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, bhi + (uint64_t)(kk * 2), id, sfa, sfb,
-                              (ks | kk) != 0);
-                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, blo + (uint64_t)(kk * 2), id, sfa, sfb, 1u);
-                }
-              } else {
-                const uint64_t bdesc = smem_desc_kmajor_sw128(tbase);
-                const uint32_t a_tmem = tmem + kACol0 + s * (kBK / 2);
-#pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                  mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
-                              (ks | kk) != 0);
-              }
-              mma_commit(smem_u32(&bar->empty[s]));
-              if (++s == kStages) { s = 0; ph ^= 1; }
-            }
-            if (ok) mma_commit(smem_u32(&bar->acc_full[acc]));
-            continue;
-          }
-          // Two k-steps per round: both stages are waited for first, then their eight MMAs
-          // go out back to back (the issuing thread blocks while the tensor pipe is busy, so
-          // the bookkeeping between rounds is the only gap the pipe can see).
-          for (int ks = 0; ks < nk; ks += 2) {
-            const bool two = ks + 1 < nk;
-            const int s1 = (s + 1 == kStages) ? 0 : s + 1;
-            const uint32_t ph1 = (s + 1 == kStages) ? (ph ^ 1) : ph;
-            if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort) ||
-                (two && !mbar_wait(smem_u32(&bar->full[s1]), ph1, err, 0x301, s_abort))) {
+          // one k-step per round: wait for its stage, issue its MMAs, release it on completion
+          const int npad = (tl.n_valid + 15) & ~15;
+          for (int ks = 0; ks < nk; ++ks) {
+            if (!mbar_wait(smem_u32(&bar->full[s]), ph, err, 0x301, s_abort)) {
               ok = false;
               break;
             }
             tc_fence_after();
+            const uint32_t tbase = tok_base + s * kTokBytes;
             if (BS) {
-              // per 32-element block: the hi part, then the lo part accumulated on top, both
-              // with the stage's scale factors (byte kk of its scale columns)
-              const int npad = (tl.n_valid + 15) & ~15;
+              const uint64_t bhi = smem_desc_kmajor_sw64(tbase);
+              const uint64_t blo = smem_desc_kmajor_sw64(tbase + kTokBytes / 2);
+              const uint32_t a_tmem = tmem + kACol0 + s * kAColsBS;
+              const uint32_t sfa = tmem + kSfaCol0 + s * 4, sfb = tmem + kSfbCol0 + s * 8;
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                if (h == 1 && !two) break;
-                const int st = h ? s1 : s;
-                const uint32_t tbase = tok_base + st * kTokBytes;
-                const uint64_t bhi = smem_desc_kmajor_sw64(tbase);
-                const uint64_t blo = smem_desc_kmajor_sw64(tbase + kTokBytes / 2);
-                const uint32_t a_tmem = tmem + kACol0 + st * kAColsBS;
-                const uint32_t sfa = tmem + kSfaCol0 + st * 4, sfb = tmem + kSfbCol0 + st * 8;
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                  const uint32_t id = idesc_mxf4a_m128(npad, (uint32_t)kk);
-                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, bhi + (uint64_t)(kk * 2), id, sfa, sfb,
-                              (ks | h | kk) != 0);
-                  mma_mxf8_ts(d_tmem, a_tmem + kk * 8, blo + (uint64_t)(kk * 2), id, sfa, sfb, 1u);
-                }
-                mma_commit(smem_u32(&bar->empty[st]));
+              for (int kk = 0; kk < 2; ++kk) {
+                const uint32_t id = idesc_mxf4a_m128(npad, (uint32_t)kk);
+                mma_mxf8_ts(d_tmem, a_tmem + kk * 8, bhi + (uint64_t)(kk * 2), id, sfa, sfb,
+                            (ks | kk) != 0);
+                mma_mxf8_ts(d_tmem, a_tmem + kk * 8, blo + (uint64_t)(kk * 2), id, sfa, sfb, 1u);
               }
             } else {
-              const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + s * kTokBytes);
+              const uint64_t bdesc = smem_desc_kmajor_sw128(tbase);
               const uint32_t a_tmem = tmem + kACol0 + s * (kBK / 2);
 #pragma unroll
               for (int kk = 0; kk < kBK / 16; ++kk)
                 mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
                             (ks | kk) != 0);
-              mma_commit(smem_u32(&bar->empty[s]));
             }
-            if (two) {
-              if (!BS) {
-                const uint64_t bdesc = smem_desc_kmajor_sw128(tok_base + s1 * kTokBytes);
-                const uint32_t a_tmem = tmem + kACol0 + s1 * (kBK / 2);
-#pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                  mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)(kk * 2), idesc, 1u);
-                mma_commit(smem_u32(&bar->empty[s1]));
-              }
-              s = (s1 + 1 == kStages) ? 0 : s1 + 1;
-              ph = (s1 + 1 == kStages) ? (ph1 ^ 1) : ph1;
-            } else {
-              s = s1;
-              ph = ph1;
-            }
+            mma_commit(smem_u32(&bar->empty[s]));
+            if (++s == kStages) { s = 0; ph ^= 1; }
           }
           if (ok) mma_commit(smem_u32(&bar->acc_full[acc]));
         }
@@ -465,8 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================ converters ====================================
     if (kRegsConv < kLaunchRegs) setmaxnreg_dec<kRegsConv>();
     // Converter warp c (0..7) serves TMEM lane quarter q = warp % 4.  A tile's k-steps are
-    // converted in pairs (2u, 2u+1), the pairs the MMA issuer waits for and issues together;
-    // the two warps of a quarter take alternate pairs (running pair index parity = c / 4).
+    // converted in pairs (2u, 2u+1) that share their scale set-up; the two warps of a quarter
+    // take alternate pairs (running pair index parity = c / 4) and publish each k-step as soon
+    // as it is stored.
     const int q = warp & 3;
     const int cidx = warp - 4;
     const int par = cidx >> 2;
@@ -610,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (active) tmem_st16(tmem + lanes + kACol0 + sa * kAColsBS, out16);
             tmem_st1(tmem + lanes + kSfaCol0 + sa * 4 + q, sfa1);
             tmem_st8(tmem + lanes + kSfbCol0 + sa * 8, sfb8);
-            if (kStageIssue) publish_stage(ga + h, true);
+            publish_stage(ga + h, true);
             continue;
           }
           uint32_t out[32];
@@ -667,23 +602,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           if (active) tmem_st32(tmem + lanes + kACol0 + sa * (kBK / 2), out);
-          if (kStageIssue) publish_stage(ga + h, active);
+          publish_stage(ga + h, active);
         }
         if (!ok) break;
-        if (kStageIssue) continue;
-        if (active || BS) tmem_wait_st();
-        tc_fence_before();
-        // packed bytes consumed and A stages written: release the weight stages and publish
-        // the A stages (this also orders the pair's reads of cw before the next pair's writes)
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(smem_u32(&bar->w_empty[ga % kWStages]));
-          mbar_arrive(smem_u32(&bar->full[ga % kStages]));
-          if (two) {
-            mbar_arrive(smem_u32(&bar->w_empty[(ga + 1) % kWStages]));
-            mbar_arrive(smem_u32(&bar->full[(ga + 1) % kStages]));
-          }
-        }
       }
       if (!ok) break;
       __syncwarp();
