@@ -90,7 +90,7 @@ constexpr int kSfbCols = kBN / 32;
 constexpr int kSfbCol0 = kSfaCol0 + kStages * 4;
 static_assert(kSfbCol0 + kStages * 8 <= kTmemCols, "TMEM budget (block-scaled)");
 static_assert(kSfbCols <= 8, "scale-factor columns of the token tile");
-static_assert(kBN % 32 == 0 && kBN <= 256, "token tile");
+static_assert(kBN % 64 == 0 && kBN <= 256, "token tile (whole pairs of 32-column chunks)");
 static_assert(wstages<false>() % 2 == 0 && wstages<true>() % 2 == 0 && kStages % 2 == 0,
               "ring depths must be even");
 
@@ -647,16 +647,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // down and dx store exactly these bf16 values; gate_up evaluates the GLU on them
         // (h rounded to bf16, as the eager bf16 model holds it).
         uint32_t pk[kBN / 32][16];
+        // two chunks per TMEM round trip (the release waits for all of them)
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 0; c < kBN / 32; c += 2) {
           if (32 * c < tl.n_valid) {
-            uint32_t r[32];
-            tmem_ld32(acc_tmem + 32 * c, r);
+            uint32_t r0[32], r1[32];
+            tmem_ld32(acc_tmem + 32 * c, r0);
+            tmem_ld32(acc_tmem + 32 * (c + 1), r1);
             tmem_wait_ld();
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj)
-              pk[c][jj] = pack_bf16x2(__uint_as_float(r[2 * jj]) + bias_f,
-                                      __uint_as_float(r[2 * jj + 1]) + bias_f);
+            for (int jj = 0; jj < 16; ++jj) {
+              pk[c][jj] = pack_bf16x2(__uint_as_float(r0[2 * jj]) + bias_f,
+                                      __uint_as_float(r0[2 * jj + 1]) + bias_f);
+              pk[c + 1][jj] = pack_bf16x2(__uint_as_float(r1[2 * jj]) + bias_f,
+                                          __uint_as_float(r1[2 * jj + 1]) + bias_f);
+            }
           }
         }
         tc_fence_before();
