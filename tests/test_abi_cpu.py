@@ -62,6 +62,15 @@ def test_unknown_gate_up_format_is_rejected(L):
         assert L.lib.mxfp4_moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == want, fmt
 
 
+def test_dims_struct_matches_header():
+    """The ctypes mirror lists the header struct's fields in order."""
+    from mxfp4_quantized_moe_b200 import _lib
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct \{([^}]*)\} mxfp4_moe_dims;", src).group(1)
+    names = re.findall(r"(\w+)\s*[,;]", body)
+    assert names == [f[0] for f in _lib.Dims._fields_]
+
+
 def test_error_codes_match_header(L):
     src = open(HEADER).read()
     codes = dict(re.findall(r"#define (MXFP4_MOE_\w+) \(?(-?\d+)\)?", src))

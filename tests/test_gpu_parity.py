@@ -229,6 +229,13 @@ def test_small_token_gpt_oss_20b_every_token(moe, T):
     check_all(got, ref)
 
 
+def test_small_token_skewed_gpt_oss_20b_every_token(moe):
+    """T=512 with Zipf-skewed routing at gpt-oss-20b widths, every token: hot experts with
+    several hundred rows (two or more token tiles) beside cold ones holding a few rows."""
+    got, ref = run_block(moe, 512, 2880, 2880, 32, 4, seed=41, zipf_s=1.2)
+    check_all(got, ref)
+
+
 def test_expert_gradient_is_not_silent(moe):
     """The pages' silent-gradient trap: dX must carry the expert path (not be zero)."""
     got, ref = run_block(moe, 16, 64, 64, 4, 2, seed=12)
