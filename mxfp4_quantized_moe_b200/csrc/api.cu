@@ -39,7 +39,7 @@ WsLayout ws_layout(const mxfp4_moe_dims& d) {
   L.perm = o;     o = up(o + 4 * A);                 // sorted row -> slot
   L.inv = o;      o = up(o + 4 * A);                 // slot -> sorted row
   L.w_row = o;    o = up(o + 4 * A);                 // routing weight of each sorted row
-  L.blk_hist = o; o = up(o + 4ull * moe::route_blocks(d.T) * d.E);
+  L.blk_hist = o; o = up(o + 4 * moe::route_scratch_words(d.T, d.E));  // routing scratch
   L.sfb = o;      o = up(o + A * sfb_stride(d.H));     // activation scales (gate_up)
   L.dgu = o;      o = up(o + 4 * A * d.I);           // saved GLU derivative factors (bf16 pairs)
   L.act = o;      o = up(o + 2 * A * d.I);           // act [A][I] (the down GEMM's input)
@@ -259,6 +259,7 @@ int mxfp4_moe_forward(const mxfp4_moe_dims* d, const mxfp4_moe_weights* w, const
   uint16_t* rows = at<uint16_t>(ws, L.rows);
 
   MOE_LAUNCH("router_topk", moe::launch_router_topk(logits, T, E, k, idx, wr, blk_hist, topk_idx, topk_w, st));
+  MOE_LAUNCH("seg_scan", moe::launch_seg_scan(T, E, blk_hist, st));
   MOE_LAUNCH("build_perm", moe::launch_build_perm(idx, wr, T, E, k, blk_hist, off, perm, inv, w_row, err, st));
   const bool bs = d->gate_up_format == MXFP4_MOE_GATE_UP_BLOCK_SCALED;
   // Xp in expert-sorted order: bf16 rows (in `rows`, which the down GEMM overwrites with y), or

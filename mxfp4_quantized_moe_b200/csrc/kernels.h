@@ -50,17 +50,22 @@ cudaError_t launch_grouped_gemm(int epi, bool transposed_scales, const void* tok
 // dynamic shared memory of a launch (sfb_stride: 0 for the bf16 form)
 size_t grouped_gemm_smem_bytes(int K, int sfb_stride);
 
-// Tokens are routed in blocks of a fixed size; blk_hist holds route_blocks(T) x E counts.
+// Tokens are routed in segments of a fixed size; the routing scratch holds
+// route_scratch_words(T, E) int32: the segments' expert histograms [route_blocks(T)][E], their
+// exclusive scans over the segments [route_blocks(T)][E] and the column totals [E].
 int route_blocks(int T);
-// top-k + softmax over the k selected logits; idx/w in slot order (t*k + j), per-block
-// expert histograms in blk_hist [route_blocks(T)][E]
+size_t route_scratch_words(int T, int E);
+// top-k + softmax over the k selected logits; idx/w in slot order (t*k + j), the segments'
+// expert histograms in the scratch
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
-                               int32_t* blk_hist, int32_t* user_idx, float* user_w,
+                               int32_t* scratch, int32_t* user_idx, float* user_w,
                                cudaStream_t st);
-// stable expert sort of the slots: off[E+1], perm[row] = slot, inv[slot] = row,
-// w_row[row] = w[slot]
+// the segments' histograms scanned over the segments, one block per expert column
+cudaError_t launch_seg_scan(int T, int E, int32_t* scratch, cudaStream_t st);
+// stable expert sort of the slots, one block per segment: off[E+1], perm[row] = slot,
+// inv[slot] = row, w_row[row] = w[slot]
 cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, int k,
-                              const int32_t* blk_hist, int32_t* off, int32_t* perm, int32_t* inv,
+                              const int32_t* scratch, int32_t* off, int32_t* perm, int32_t* inv,
                               float* w_row, int* err, cudaStream_t st);
 // dst[r] = src[perm[r] / k] for every expert-sorted row r.  With `dot_w` (the backward's
 // gather of dY), `dst` first holds the forward's expert outputs y in sorted order, which are

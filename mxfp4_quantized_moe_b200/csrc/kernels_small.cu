@@ -15,134 +15,158 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---------------------------------------------------------------------------------------
 // Router: top-k over the E logits of a token (largest first, equal logits -> lower expert
-// index) and softmax over the k selected.  One warp per token: lane l holds logits l, l+32,
-// ... (E <= 256); each of the k rounds is a lane-local best followed by a five-step
-// butterfly argmax.  Lane j keeps selection j and adds it to the expert histogram of the
-// token's 128-token segment (blk_hist[t / 128][e], zeroed before the launch), which lets the
-// permutation kernel place every segment's slots without another pass over the routing.
+// index) and softmax over the k selected.  One warp per token, one block per 32-token
+// segment.  Lane l holds logits l, l+32, ... (NG = ceil(E/32) of them) as order-preserving
+// 32-bit keys; each of the k rounds takes the lane's best remaining key, the warp's largest
+// key (one redux.sync) and the lowest expert index among the lanes holding it (a second).
+// NaN logits never win (they rank as -inf), and -0 ranks with +0.  Lane j keeps selection j
+// and counts it in the segment's expert histogram in shared memory, which the block stores as
+// row t / 32 of `hist`; the segment scan and the permutation kernel place every segment's
+// slots from these rows without another pass over the routing.
 // Source: the top-k router of the eager expert loop ("Add MXFP4 training support via a
 // dequantize-on-the-fly fallback", section "What this does"); softmax over the k values.
 // ---------------------------------------------------------------------------------------
-constexpr int kRouteThreads = 256;
-constexpr int kRouteTokens = 128;  // tokens per histogram segment / permutation block
+constexpr int kRouteTokens = 32;                  // tokens per histogram segment
+constexpr int kRouteThreads = 32 * kRouteTokens;  // one warp per token
+constexpr int kPermThreads = 256;                 // permutation block (one segment)
+constexpr int kScanThreads = 512;                 // segment scan (one expert column)
 
-__device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
-  return v > bv || (v == bv && i < bi);
+// float -> unsigned key with the same order (x assumed not NaN); the inverse below
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t b = __float_as_uint(x);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+template <int NG>
 __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(
     const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
-    float* __restrict__ w, int32_t* __restrict__ blk_hist, int32_t* __restrict__ user_idx,
+    float* __restrict__ w, int32_t* __restrict__ hist, int32_t* __restrict__ user_idx,
     float* __restrict__ user_w) {
-  const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * kRouteThreads + threadIdx.x) >> 5;
-  if (t >= T) return;
-  const float* row = logits + (size_t)t * E;
-  float v[8];
-  uint32_t taken = 0;  // bit i: expert lane + 32 i already selected (or absent)
+  __shared__ int s_hist[256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += kRouteThreads) s_hist[e] = 0;
+  __syncthreads();
+  const int seg = blockIdx.x;
+  const int t = seg * kRouteTokens + warp;
+  if (t < T) {  // warp-uniform
+    const float* row = logits + (size_t)t * E;
+    uint32_t key[NG];  // 0: absent or already selected (every present logit's key is larger)
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    const float x = (e < E) ? __ldg(row + e) : -INFINITY;
-    v[i] = (x != x) ? -INFINITY : x;  // a NaN logit is never preferred
-    if (e >= E) taken |= 1u << i;
-  }
-  float m0 = 0.f, zsum = 0.f;
-  float myz = 0.f;  // selection `lane` (k <= 32); lane j % 32 parks selections j >= 32 in
-  int myi = 0;      // idx / w until the softmax denominator is known
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7FFFFFFF;
+    for (int i = 0; i < NG; ++i) {
+      const int e = lane + 32 * i;
+      float x = (e < E) ? __ldg(row + e) : 0.f;
+      x = (x != x) ? -INFINITY : x + 0.f;  // NaN ranks as -inf; -0 + 0 = +0
+      key[i] = (e < E) ? order_key(x) : 0u;
+    }
+    float m0 = 0.f, zsum = 0.f;
+    float myz = 0.f;  // selection `lane` (k <= 32); lane j % 32 parks selections j >= 32 in
+    int myi = 0;      // idx / w until the softmax denominator is known
+    for (int j = 0; j < k; ++j) {
+      uint32_t hk = 0;
+      int hi = 0x7FFFFFFF;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (!(taken & (1u << i)) && beats(v[i], lane + 32 * i, bv, bi)) {
-        bv = v[i];
-        bi = lane + 32 * i;
+      for (int i = 0; i < NG; ++i)  // strictly larger: the lower expert wins a tie
+        if (key[i] > hk) {
+          hk = key[i];
+          hi = lane + 32 * i;
+        }
+      const uint32_t mk = __reduce_max_sync(kFull, hk);
+      const int bi = (int)__reduce_min_sync(kFull, hk == mk ? (uint32_t)hi : 0x7FFFFFFFu);
+      if ((bi & 31) == lane) {
+#pragma unroll
+        for (int i = 0; i < NG; ++i)
+          if (i == (bi >> 5)) key[i] = 0u;
       }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float ov = __shfl_xor_sync(kFull, bv, o);
-      const int oi = __shfl_xor_sync(kFull, bi, o);
-      if (beats(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
+      const float bv = key_value(mk);
+      if (j == 0) m0 = bv;
+      const float z = __expf(bv - m0);
+      zsum += z;
+      if (lane == (j & 31)) {
+        if (j < 32) {
+          myz = z;
+          myi = bi;
+        } else {
+          w[(size_t)t * k + j] = z;
+          idx[(size_t)t * k + j] = bi;
+        }
       }
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (j == 0) m0 = bv;
-    const float z = __expf(bv - m0);
-    zsum += z;
-    if (lane == (j & 31)) {
-      if (j < 32) {
-        myz = z;
-        myi = bi;
-      } else {
-        w[(size_t)t * k + j] = z;
-        idx[(size_t)t * k + j] = bi;
-      }
+    const float inv = 1.f / zsum;
+    for (int j = lane; j < k; j += 32) {
+      const size_t o = (size_t)t * k + j;
+      const float z = (j < 32) ? myz : w[o];
+      const int e = (j < 32) ? myi : idx[o];
+      const float wj = z * inv;
+      idx[o] = e;
+      w[o] = wj;
+      if (user_idx) user_idx[o] = e;
+      if (user_w) user_w[o] = wj;
+      atomicAdd(s_hist + e, 1);
     }
   }
-  const float inv = 1.f / zsum;
-  int32_t* hist = blk_hist + (size_t)(t / kRouteTokens) * E;
-  for (int j = lane; j < k; j += 32) {
-    const size_t o = (size_t)t * k + j;
-    const float z = (j < 32) ? myz : w[o];
-    const int e = (j < 32) ? myi : idx[o];
-    const float wj = z * inv;
-    idx[o] = e;
-    w[o] = wj;
-    if (user_idx) user_idx[o] = e;
-    if (user_w) user_w[o] = wj;
-    atomicAdd(hist + e, 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kRouteThreads) hist[(size_t)seg * E + e] = s_hist[e];
+}
+
+// Exclusive scan of one expert's column of the segment histograms (block e):
+// seg_pre[s][e] = sum of hist[s'][e] over s' < s, tot[e] = the column's sum.
+__global__ void __launch_bounds__(kScanThreads) seg_scan_kernel(
+    const int32_t* __restrict__ hist, int nseg, int E, int32_t* __restrict__ seg_pre,
+    int32_t* __restrict__ tot) {
+  __shared__ int s_warp[kScanThreads / 32];
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int carry = 0;
+  for (int c = 0; c < nseg; c += kScanThreads) {
+    const int s = c + threadIdx.x;
+    const int v = s < nseg ? __ldg(hist + (size_t)s * E + e) : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int wbase = 0, chunk = 0;
+    for (int i = 0; i < kScanThreads / 32; ++i) {
+      const int x = s_warp[i];
+      wbase += (i < warp) ? x : 0;
+      chunk += x;
+    }
+    if (s < nseg) seg_pre[(size_t)s * E + e] = carry + wbase + incl - v;
+    carry += chunk;
+    __syncthreads();  // s_warp is rewritten by the next chunk
   }
+  if (threadIdx.x == 0) tot[e] = carry;
 }
 
 // ---------------------------------------------------------------------------------------
-// Stable counting sort of the A = T*k slots by expert, one block per router block.  Block b
-// sums the router blocks' histograms into (a) the expert offsets off[e] (an exclusive scan of
-// the totals) and (b) the number of expert-e slots in blocks before b; its own slots are then
-// ranked in slot order: each warp counts a contiguous share of them per expert (warp-level
-// match on the expert id), a scan over the warps gives each share's first row, and a second
-// pass assigns the rows.  perm[row] = slot, inv[slot] = row, w_row[row] = w[slot]; block 0
+// Stable counting sort of the A = T*k slots by expert, one block per routing segment.  The
+// expert offsets off[e] are the exclusive scan of the column sums over the experts; the
+// segment's first expert-e row is off[e] + seg_pre[b][e].  The block's slots are then ranked
+// in slot order: each warp counts a contiguous share of them per expert (warp-level match on
+// the expert id), a scan over the warps gives each share's first row, and a second pass
+// assigns the rows.  perm[row] = slot, inv[slot] = row, w_row[row] = w[slot]; block 0
 // publishes off[0..E].
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kRouteThreads) build_perm_kernel(
+__global__ void __launch_bounds__(kPermThreads) build_perm_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ w, int A, int E, int k,
-    const int32_t* __restrict__ blk_hist, int nblk, int32_t* __restrict__ off,
-    int32_t* __restrict__ perm, int32_t* __restrict__ inv, float* __restrict__ w_row, int* err) {
-  constexpr int kWarps = kRouteThreads / 32;
+    const int32_t* __restrict__ seg_pre, const int32_t* __restrict__ tot,
+    int32_t* __restrict__ off, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    float* __restrict__ w_row, int* err) {
+  constexpr int kWarps = kPermThreads / 32;
+  static_assert(kPermThreads >= 256, "one thread per expert (E <= 256)");
   __shared__ int s_cnt[kWarps][256];
   __shared__ int s_tot[256];
   __shared__ int s_scan[kWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
-  // (a) + (b): column sums of the [nblk][E] segment histograms; `parts` threads share each
-  // expert's column (strided over the segments), then their partial sums are added
-  __shared__ int s_part[2][kRouteThreads];
   const int e = threadIdx.x;
-  {
-    const int parts = kRouteThreads / E;  // >= 1 (E <= 256)
-    const int ex = threadIdx.x % E, part = threadIdx.x / E;
-    int bf = 0, tot = 0;
-    if (part < parts) {
-#pragma unroll 4
-      for (int bb = part; bb < nblk; bb += parts) {
-        const int c = __ldg(blk_hist + (size_t)bb * E + ex);
-        tot += c;
-        bf += (bb < b) ? c : 0;
-      }
-    }
-    s_part[0][threadIdx.x] = bf;
-    s_part[1][threadIdx.x] = tot;
-    __syncthreads();
-  }
-  int before = 0, total = 0;
-  if (e < E) {
-    for (int i = e; i < kRouteThreads - (kRouteThreads % E); i += E) {
-      before += s_part[0][i];
-      total += s_part[1][i];
-    }
-  }
+  const int total = (e < E) ? __ldg(tot + e) : 0;
   // exclusive scan of the totals over experts (E <= 256 = one value per thread)
   int incl = total;
 #pragma unroll
@@ -155,7 +179,7 @@ __global__ void __launch_bounds__(kRouteThreads) build_perm_kernel(
   int wbase = 0;
   for (int i = 0; i < warp; ++i) wbase += s_scan[i];
   const int off_e = wbase + incl - total;
-  if (e < E) s_tot[e] = off_e + before;  // first row of this block's expert-e slots
+  if (e < E) s_tot[e] = off_e + __ldg(seg_pre + (size_t)b * E + e);  // first row of this block's expert-e slots
   if (b == 0) {
     if (e < E) off[e] = off_e;
     if (e == E - 1) {
@@ -399,27 +423,43 @@ __global__ void combine_kernel(const uint16_t* __restrict__ rows, const int32_t*
 }
 
 // d_logits through the softmax over the k selected logits:
-// d_l[idx_j] = w_j (d_w_j - sum_i w_i d_w_i), 0 for the experts not selected.  One thread per
-// output element (token t, expert e), so that the [T][E] stores are coalesced; the k-term
-// sums are re-read from L1 by the E threads of a token.
+// d_l[idx_j] = w_j (d_w_j - sum_i w_i d_w_i), 0 for the experts not selected.  One warp per
+// token: the k selections are read once (lane j % 32 takes selection j), the sum is a warp
+// reduction, and the row of E outputs is stored by the 32 lanes together (coalesced).
 __global__ void router_backward_kernel(const int32_t* __restrict__ idx,
                                        const float* __restrict__ w,
                                        const float* __restrict__ d_topk_w, int T, int E, int k,
                                        float* __restrict__ d_logits) {
-  const size_t n = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= (size_t)T * E) return;
-  const int t = (int)(n / E), e = (int)(n % E);
+  const int lane = threadIdx.x & 31;
+  const int t = (int)(((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if (t >= T) return;  // warp-uniform
   const int32_t* it = idx + (size_t)t * k;
   const float* wt = w + (size_t)t * k;
   const float* dt = d_topk_w + (size_t)t * k;
-  float s = 0.f, out = 0.f;
-  int mine = -1;
-  for (int j = 0; j < k; ++j) {
-    s += __ldg(wt + j) * __ldg(dt + j);
-    if (__ldg(it + j) == e) mine = j;
+  // s = sum_j w_j d_w_j over the k selections (lane j % 32 takes selection j)
+  float s = 0.f;
+  for (int j = lane; j < k; j += 32) s += __ldg(wt + j) * __ldg(dt + j);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+  // lane l writes experts l, l+32, ...: the selected ones get w_j (d_w_j - s)
+  float out[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int j0 = 0; j0 < k; j0 += 32) {
+    const int j = j0 + lane;
+    const int ej = j < k ? __ldg(it + j) : -1;
+    const float gj = j < k ? __ldg(wt + j) * (__ldg(dt + j) - s) : 0.f;
+    const int n = min(32, k - j0);
+    for (int q = 0; q < n; ++q) {
+      const int e = __shfl_sync(kFull, ej, q);
+      const float g = __shfl_sync(kFull, gj, q);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (e == lane + 32 * i) out[i] = g;
+    }
   }
-  if (mine >= 0) out = __ldg(wt + mine) * (__ldg(dt + mine) - s);
-  d_logits[n] = out;
+  float* dl = d_logits + (size_t)t * E;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (lane + 32 * i < E) dl[lane + 32 * i] = out[i];
 }
 
 // One thread per 8 elements (one 32-bit word of codes, a quarter of an MX block): a warp reads
@@ -487,23 +527,34 @@ __global__ void transpose_scales_kernel(const uint8_t* __restrict__ src, int R, 
 
 int route_blocks(int T) { return (T + kRouteTokens - 1) / kRouteTokens; }
 
+size_t route_scratch_words(int T, int E) { return 2 * (size_t)route_blocks(T) * E + E; }
+
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
-                               int32_t* blk_hist, int32_t* user_idx, float* user_w,
+                               int32_t* scratch, int32_t* user_idx, float* user_w,
                                cudaStream_t st) {
-  cudaError_t e = cudaMemsetAsync(blk_hist, 0, sizeof(int32_t) * (size_t)route_blocks(T) * E, st);
-  if (e != cudaSuccess) return e;
-  const int warps_per_block = kRouteThreads / 32;
-  router_topk_kernel<<<(T + warps_per_block - 1) / warps_per_block, kRouteThreads, 0, st>>>(
-      logits, T, E, k, idx, w, blk_hist, user_idx, user_w);
+  const int ng = (E + 31) / 32;
+  auto kern = ng <= 1 ? router_topk_kernel<1> : ng <= 2 ? router_topk_kernel<2>
+            : ng <= 4 ? router_topk_kernel<4> : router_topk_kernel<8>;
+  kern<<<route_blocks(T), kRouteThreads, 0, st>>>(logits, T, E, k, idx, w, scratch, user_idx,
+                                                   user_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_seg_scan(int T, int E, int32_t* scratch, cudaStream_t st) {
+  const int nseg = route_blocks(T);
+  int32_t* seg_pre = scratch + (size_t)nseg * E;
+  seg_scan_kernel<<<E, kScanThreads, 0, st>>>(scratch, nseg, E, seg_pre, seg_pre + (size_t)nseg * E);
   return cudaGetLastError();
 }
 
 cudaError_t launch_build_perm(const int32_t* idx, const float* w, int T, int E, int k,
-                              const int32_t* blk_hist, int32_t* off, int32_t* perm, int32_t* inv,
+                              const int32_t* scratch, int32_t* off, int32_t* perm, int32_t* inv,
                               float* w_row, int* err, cudaStream_t st) {
-  const int nblk = route_blocks(T);
-  build_perm_kernel<<<nblk, kRouteThreads, 0, st>>>(idx, w, T * k, E, k, blk_hist, nblk, off, perm,
-                                                    inv, w_row, err);
+  const int nseg = route_blocks(T);
+  const int32_t* seg_pre = scratch + (size_t)nseg * E;
+  build_perm_kernel<<<nseg, kPermThreads, 0, st>>>(idx, w, T * k, E, k, seg_pre,
+                                                   seg_pre + (size_t)nseg * E, off, perm, inv,
+                                                   w_row, err);
   return cudaGetLastError();
 }
 
@@ -535,7 +586,7 @@ cudaError_t launch_combine(const uint16_t* rows, const int32_t* inv, const float
 cudaError_t launch_router_backward(const int32_t* idx, const float* w, const float* d_topk_w,
                                    int T, int E, int k, float* d_logits, cudaStream_t st) {
   if (!d_logits) return cudaSuccess;
-  const size_t n = (size_t)T * E;
+  const size_t n = (size_t)T * 32;  // one warp per token
   router_backward_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(idx, w, d_topk_w, T, E, k,
                                                                      d_logits);
   return cudaGetLastError();

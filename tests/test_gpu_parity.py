@@ -184,6 +184,34 @@ def test_router_ties_and_topk_exact(moe):
     np.testing.assert_allclose(tw.cpu().numpy(), wr, rtol=2e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("E,k", [(256, 40), (128, 4), (40, 33)])
+def test_router_signed_zeros_infinities_and_wide_k(moe, E, k):
+    """Top-k against the oracle's stable sort where the ranking is delicate: +0 and -0 tie (the
+    lower expert wins), -inf logits rank last, negative logits, every group of 32 experts of a
+    lane occupied (E = 256), and more than 32 selections per token (k = 40 and 33)."""
+    T, H, I = 64, 64, 64
+    inp = inputs.make_layer(T, H, I, E, k, seed=21)
+    lg = inp["logits"].clone()
+    lg[0] = 0.0
+    lg[0, 1::2] = -0.0                                   # +0 / -0 alternate: all tie
+    lg[1] = -torch.arange(E, dtype=torch.float32)       # strictly decreasing from 0
+    lg[1, 3] = -0.0                                      # -0 ties with expert 0's +0
+    lg[2] = float("-inf")
+    lg[2, E - 1] = -1e30                                 # one finite logit, then -inf ties
+    lg[3, ::3] = float("-inf")
+    lg[4] = torch.where(torch.arange(E) % 5 == 0, 2.5, -2.5)  # five-way groups of ties
+    shape = moe.MoeShape(T, H, I, E, k)
+    w = moe.weights_to(inp, "cuda")
+    ws = moe.alloc_workspace(shape)
+    ti = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    moe.forward(shape, w, inp["x"].cuda(), lg.cuda(), ws, topk_idx=ti, topk_w=tw)
+    assert moe.device_check(ws) == (0, 0)
+    idx, wr = O.route(lg.numpy(), k)
+    assert np.array_equal(ti.cpu().numpy(), idx)
+    np.testing.assert_allclose(tw.cpu().numpy(), wr, rtol=2e-6, atol=1e-7)
+
+
 # ------------------------------------------------------------------ whole block -------
 def test_tiny_workload_full_parity(moe):
     wl = inputs.WORKLOADS["tiny-moe-T64-H256-E8-k2"]
@@ -362,13 +390,14 @@ def _sfb_natural(sfb):
 
 def _ws_offsets(T, E, k, H=None, I=None):
     """Offsets of the regions of the forward's workspace (the library's layout: each region
-    starts 256-byte aligned, in the order error word, offsets, idx, w, perm, inv, w_row, router
-    block histograms, activation scales, GLU factors, act, dH, rows)."""
+    starts 256-byte aligned, in the order error word, offsets, idx, w, perm, inv, w_row, routing
+    scratch (the 32-token segments' expert histograms, their scans over the segments and the
+    column totals), activation scales, GLU factors, act, dH, rows)."""
     def up(v):
         return (v + 255) // 256 * 256
     A = T * k
     sizes = [("err", 16), ("off", 4 * (E + 1)), ("idx", 4 * A), ("w", 4 * A), ("perm", 4 * A),
-             ("inv", 4 * A), ("w_row", 4 * A), ("blk_hist", 4 * (-(-T // 128)) * E)]
+             ("inv", 4 * A), ("w_row", 4 * A), ("blk_hist", 4 * (2 * (-(-T // 32)) * E + E))]
     if H is not None:
         sizes += [("sfb", A * _sfb_stride(H)), ("dgu", 4 * A * I), ("act", 2 * A * I),
                   ("dh", 2 * A * max(2 * I, H)), ("rows", 2 * A * H)]
