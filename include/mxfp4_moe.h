@@ -250,6 +250,38 @@ MXFP4_MOE_API int mxfp4_moe_grouped_matmul(int32_t E, int32_t N, int32_t K, int3
                                            int32_t transposed, uint16_t* out, int32_t* err_word,
                                            void* stream);
 
+/* The residual stream between stacked blocks, the caller's side of the block boundary, in one
+ * kernel.  Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", section
+ * "What this does" (decoder layers around the MoE block, trained with gradient
+ * checkpointing: residual stream and router linear); the fusion has no counterpart there.
+ *   x_out[t][h]  = bf16(x[t][h] + y[t][h])          fp32 sum rounded once (round to nearest
+ *                                                   even); only when y is not NULL
+ *   logits[t][e] = sum_h xs[t][h] * w_r[h][e] + b_r[e]   fp32 accumulation of the bf16
+ *                                                   products, xs = x_out (y given) or x
+ *                                                   (y NULL); only when logits is not NULL
+ *   x, y, x_out  bf16 [T][H] DEVICE, 16-byte aligned; x_out NULL exactly when y is NULL
+ *   w_r          bf16 [H][E] DEVICE, 16-byte aligned (the router linear), required with logits
+ *   b_r          bf16 [E] DEVICE or NULL (no bias)
+ *   logits       fp32 [T][E] DEVICE or NULL
+ * T >= 0, H a multiple of 32, 1 <= E <= 256; at least one of y and logits.  x_out must not
+ * overlap x or y.  Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_residual_router(int32_t T, int32_t H, int32_t E, const uint16_t* x,
+                                            const uint16_t* y, const uint16_t* w_r,
+                                            const uint16_t* b_r, uint16_t* x_out,
+                                            float* logits, void* stream);
+
+/* The residual stream's gradient through one stacked block, in one kernel (source as for
+ * mxfp4_moe_residual_router):
+ *   g_out[t][h] = bf16(g[t][h] + dx[t][h] + sum_e d_logits[t][e] * w_r[h][e])
+ * in fp32 (the sum over e in ascending order, then g + dx + that sum), rounded once.
+ *   g, dx, g_out  bf16 [T][H] DEVICE, 16-byte aligned; g_out may be g itself
+ *   d_logits      fp32 [T][E] DEVICE (mxfp4_moe_backward_input's router gradient)
+ *   w_r           bf16 [H][E] DEVICE, 16-byte aligned
+ * T >= 0, H a multiple of 32, 1 <= E <= 256.  Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+MXFP4_MOE_API int mxfp4_moe_grad_chain(int32_t T, int32_t H, int32_t E, const uint16_t* g,
+                                       const uint16_t* dx, const float* d_logits,
+                                       const uint16_t* w_r, uint16_t* g_out, void* stream);
+
 /* Standalone dequantization (diagnostics and tests): rows of packed MXFP4 -> bf16.
  * Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback", section "What this does" (`_dequantize_weights`); OCP MX v1.0.
  *   blocks uint8 [rows][K/2], scales uint8 [rows][K/32], out bf16 [rows][K]; K multiple of 32.

@@ -66,6 +66,10 @@ SIGNATURES = {
                                                 ctypes.c_int32, _vp, _vp, _vp, _vp, ctypes.c_int32,
                                                 _vp, _vp, _vp]),
     "mxfp4_moe_dequantize": (ctypes.c_int, [_vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp]),
+    "mxfp4_moe_residual_router": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mxfp4_moe_grad_chain": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                            _vp, _vp, _vp, _vp, _vp, _vp]),
     "mxfp4_moe_check": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "mxfp4_moe_selftest_wait_timeout": (ctypes.c_int, [_vp, ctypes.c_size_t, _vp]),
     "mxfp4_moe_interleave_gate_up": (ctypes.c_int, [ctypes.POINTER(Dims), _vp, _vp, _vp, _vp, _vp,

@@ -23,7 +23,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmxfp4_moe.so")
 LIB_DEBUG = os.path.join(HERE, "libmxfp4_moe_debug.so")
 SOURCES = ["csrc/api.cu", "csrc/grouped_gemm.cu", "csrc/kernels_small.cu",
-           "csrc/forward_static.cu", "csrc/selftest.cu"]
+           "csrc/forward_static.cu", "csrc/selftest.cu", "csrc/residual_router.cu"]
 DEPS = SOURCES + ["csrc/common.cuh", "csrc/kernels.h", "csrc/aux_kernels.h"]
 
 

@@ -389,6 +389,44 @@ int mxfp4_moe_interleave_gate_up(const mxfp4_moe_dims* d, const uint8_t* stacked
   return MXFP4_MOE_OK;
 }
 
+int mxfp4_moe_residual_router(int32_t T, int32_t H, int32_t E, const uint16_t* x,
+                              const uint16_t* y, const uint16_t* w_r, const uint16_t* b_r,
+                              uint16_t* x_out, float* logits, void* stream) {
+  if (T < 0 || H < 32 || H % 32 || E < 1 || E > 256 || !x || !aligned16(x))
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  if (!y && !logits) return MXFP4_MOE_ERR_INVALID_ARG;
+  if ((y == nullptr) != (x_out == nullptr)) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (y && (!aligned16(y) || !aligned16(x_out))) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (logits && (!w_r || !aligned16(w_r))) return MXFP4_MOE_ERR_INVALID_ARG;
+  if (x_out) {  // x_out overlapping x or y would be read after being written
+    const size_t n = 2 * (size_t)T * H;
+    auto overlaps = [n](const void* a, const void* b) {
+      const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+      return pa < pb + n && pb < pa + n;
+    };
+    if (T > 0 && (overlaps(x_out, x) || overlaps(x_out, y))) return MXFP4_MOE_ERR_INVALID_ARG;
+  }
+  const int rc = check_device(nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_LAUNCH("residual_router",
+             moe::launch_residual_router(T, H, E, x, y, w_r, b_r, x_out, logits, st));
+  return MXFP4_MOE_OK;
+}
+
+int mxfp4_moe_grad_chain(int32_t T, int32_t H, int32_t E, const uint16_t* g, const uint16_t* dx,
+                         const float* d_logits, const uint16_t* w_r, uint16_t* g_out,
+                         void* stream) {
+  if (T < 0 || H < 32 || H % 32 || E < 1 || E > 256 || !g || !dx || !d_logits || !w_r || !g_out ||
+      !aligned16(g) || !aligned16(dx) || !aligned16(w_r) || !aligned16(g_out))
+    return MXFP4_MOE_ERR_INVALID_ARG;
+  const int rc = check_device(nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_LAUNCH("grad_chain", moe::launch_grad_chain(T, H, E, g, dx, d_logits, w_r, g_out, st));
+  return MXFP4_MOE_OK;
+}
+
 int mxfp4_moe_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < 16 || !aligned16(ws)) return MXFP4_MOE_ERR_INVALID_ARG;
   const int rc = check_device(nullptr);

@@ -171,6 +171,53 @@ def interleave_gate_up(shape: MoeShape, blocks: torch.Tensor, scales: torch.Tens
     return ob, os_, obias
 
 
+def residual_router(x: torch.Tensor, y: torch.Tensor | None, w_r: torch.Tensor | None,
+                    b_r: torch.Tensor | None = None, x_out: torch.Tensor | None = None,
+                    logits: torch.Tensor | None = None, stream=None):
+    """The residual stream between stacked blocks in one kernel: x_out = bf16(x + y) when y is
+    given, and logits = (x_out or x) W_r + b_r in fp32 when w_r is given.  Returns
+    (x_out or None, logits or None)."""
+    T, H = x.shape
+    if x.dtype != torch.bfloat16 or (y is not None and (y.shape != x.shape or y.dtype != x.dtype)):
+        raise ValueError("x and y must be bf16 [T, H]")
+    E = w_r.shape[1] if w_r is not None else 1
+    if w_r is not None:
+        if w_r.shape != (H, E) or w_r.dtype != torch.bfloat16:
+            raise ValueError("w_r must be bf16 [H, E]")
+        if b_r is not None and (b_r.shape != (E,) or b_r.dtype != torch.bfloat16):
+            raise ValueError("b_r must be bf16 [E]")
+        if logits is None:
+            logits = torch.empty(T, E, dtype=torch.float32, device=x.device)
+    else:
+        logits = None
+    if y is not None and x_out is None:
+        x_out = torch.empty_like(x)
+    if y is None:
+        x_out = None
+    check(lib.mxfp4_moe_residual_router(T, H, E, _ptr(x), _ptr(y), _ptr(w_r), _ptr(b_r),
+                                        _ptr(x_out), _ptr(logits), _stream(stream)),
+          "mxfp4_moe_residual_router")
+    return x_out, logits
+
+
+def grad_chain(g: torch.Tensor, dx: torch.Tensor, d_logits: torch.Tensor, w_r: torch.Tensor,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bf16(g + dx + d_logits W_r^T) in fp32, one kernel (out may be g itself)."""
+    T, H = g.shape
+    E = w_r.shape[1]
+    if g.dtype != torch.bfloat16 or dx.shape != g.shape or dx.dtype != g.dtype:
+        raise ValueError("g and dx must be bf16 [T, H]")
+    if d_logits.shape != (T, E) or d_logits.dtype != torch.float32:
+        raise ValueError("d_logits must be fp32 [T, E]")
+    if w_r.shape != (H, E) or w_r.dtype != torch.bfloat16:
+        raise ValueError("w_r must be bf16 [H, E]")
+    if out is None:
+        out = torch.empty_like(g)
+    check(lib.mxfp4_moe_grad_chain(T, H, E, _ptr(g), _ptr(dx), _ptr(d_logits), _ptr(w_r),
+                                   _ptr(out), _stream(stream)), "mxfp4_moe_grad_chain")
+    return out
+
+
 def selftest_wait_timeout(ws: torch.Tensor, stream=None) -> None:
     """Enqueue the failure-detection self-test on `ws` (first 16 bytes zero); read the outcome
     with device_check(ws): (MXFP4_MOE_ERR_DEVICE_TIMEOUT, 0xF00) after about one second."""

@@ -3,19 +3,21 @@
     x_{l+1} = x_l + MoE_l(x_l, logits_l),   logits_l = x_l W_r^l + b_r^l   (fp32)
 
 The blocks are the library's entry points (mxfp4_moe_forward / mxfp4_moe_backward_input);
-this module is the caller around them: the router linear, the residual add and the router's
-input gradient (d_logits W_r^T) are the caller's side of the block boundary and run as
-plain torch ops.  The backward is activation checkpointing at block granularity: the
-forward keeps only each block's input x_l (bf16); the backward re-runs block l's forward
-from x_l to refill the one shared workspace, then runs its input-gradient backward, so at
-most one block's transients are alive at any time.
+the caller's side of the block boundary is two more of its kernels: mxfp4_moe_residual_router
+forms x_{l+1} = bf16(x_l + y_l) and the next block's logits from one read of x_l and y_l, and
+mxfp4_moe_grad_chain forms g_l below.  The backward is activation checkpointing at block
+granularity: the forward keeps only each block's input x_l (bf16); the backward re-runs
+block l's forward from x_l to refill the one shared workspace, then runs its input-gradient
+backward, so at most one block's transients are alive at any time.
 
 Chain rule per block (g_{l+1} = dL/dx_{l+1}):
     g_l = g_{l+1} + dX_moe_l + d_logits_l (W_r^l)^T
 with dX_moe_l and d_logits_l returned by the block's backward for upstream gradient g_{l+1}.
 Sums are taken in fp32 and rounded to bf16 once per block, like the residual stream.
 
-The block functions are injectable so that the chaining itself can be checked on the CPU
+The forward checkpoints each block's input x_l together with its logits_l (T x E fp32, a
+few MB a block), so the recompute needs no router call.  The block functions and the two
+caller-side steps are injectable, so that the chaining itself can be checked on the CPU
 against an fp64 reference without a GPU.
 
 Source: "Add MXFP4 training support via a dequantize-on-the-fly fallback" (the MoE block of
@@ -42,46 +44,26 @@ class StackBlock:
     b_r: torch.Tensor
 
 
-def _wide(t: torch.Tensor) -> torch.Tensor:
-    """16-bit floats widen to fp32 for arithmetic; wider types stay as they are."""
-    return t.float() if t.dtype in (torch.bfloat16, torch.float16) else t
-
-
-def router_logits(x: torch.Tensor, w_r: torch.Tensor, b_r: torch.Tensor) -> torch.Tensor:
-    """Logits of the residual stream, x W_r + b_r (the caller's router linear), in fp32 for
-    a bf16 stream.  On the GPU a bf16 stream goes through one GEMM with fp32 accumulation and
-    fp32 output (no widened copy of x)."""
-    if x.is_cuda and x.dtype == torch.bfloat16 and w_r.dtype == torch.bfloat16:
-        return torch.addmm(_wide(b_r), x, w_r, out_dtype=torch.float32)
-    return torch.addmm(_wide(b_r), _wide(x), _wide(w_r))
-
-
-def residual_add(x: torch.Tensor, y: torch.Tensor) -> torch.Tensor:
-    """x + y in fp32, rounded once to the stream's dtype (one elementwise kernel: torch adds
-    16-bit floats in fp32 and rounds the result)."""
-    return x + y if x.dtype == y.dtype else (_wide(x) + _wide(y)).to(x.dtype)
-
-
-def grad_chain(g: torch.Tensor, dx: torch.Tensor, d_logits: torch.Tensor,
-               w_r: torch.Tensor) -> torch.Tensor:
-    """g + dx + d_logits W_r^T in fp32, rounded once to g's dtype: the router path's GEMM
-    accumulates onto g (fp32), then dx is added in place."""
-    acc = torch.addmm(_wide(g), _wide(d_logits), _wide(w_r).t())
-    acc += dx
-    return acc.to(g.dtype)
-
-
 class MoeStack:
     """Forward and recompute-per-block backward over a list of blocks.
 
     `block_forward(l, x, logits) -> y` and `block_backward(l, g) -> (dx, d_logits)` default to
     the library's entry points on one shared workspace; `block_backward` sees the workspace
-    that the immediately preceding `block_forward(l, ...)` left."""
+    that the immediately preceding `block_forward(l, ...)` left.
+    `residual_router(x, y, w_r, b_r) -> (x + y or None, logits or None)` (y None: logits of
+    x; w_r None: no logits) and `grad_chain(g, dx, d_logits, w_r)` default to the library's
+    mxfp4_moe_residual_router and mxfp4_moe_grad_chain."""
 
     def __init__(self, shape, blocks: list[StackBlock], device=None,
-                 block_forward: Callable | None = None, block_backward: Callable | None = None):
+                 block_forward: Callable | None = None, block_backward: Callable | None = None,
+                 residual_router: Callable | None = None, grad_chain: Callable | None = None):
         self.shape = shape
         self.blocks = blocks
+        if residual_router is None or grad_chain is None:
+            from . import moe
+            self._moe = moe
+        self.residual_router = residual_router or self._lib_residual_router
+        self.grad_chain = grad_chain or self._lib_grad_chain
         if block_forward is None or block_backward is None:
             from . import moe
             self._moe = moe
@@ -105,17 +87,28 @@ class MoeStack:
                                                d_topk_w=self._dtw, d_logits=self._dl)
         return dx, dl, dtw
 
+    def _lib_residual_router(self, x, y, w_r, b_r):
+        return self._moe.residual_router(x, y, w_r, b_r)
+
+    def _lib_grad_chain(self, g, dx, d_logits, w_r):
+        return self._moe.grad_chain(g, dx, d_logits, w_r)
+
     # ---- the stack -----------------------------------------------------------------------
     def forward(self, x: torch.Tensor, tap: Callable | None = None):
-        """Returns (x_L, saved block inputs).  `tap(l, dict)` sees each block's x, logits, y."""
+        """Returns (x_L, saved), saved[l] = (x_l, logits_l) for the recompute.  `tap(l, dict)`
+        sees each block's x, logits, y."""
         saved = []
-        for l, b in enumerate(self.blocks):
-            saved.append(x)
-            logits = router_logits(x, b.w_r, b.b_r)
+        first = self.blocks[0]
+        logits = self.residual_router(x, None, first.w_r, first.b_r)[1]
+        for l in range(len(self.blocks)):
+            saved.append((x, logits))
             y = self.block_forward(l, x, logits)
             if tap is not None:
                 tap(l, {"x": x, "logits": logits, "y": y})
-            x = residual_add(x, y)
+            nxt = self.blocks[l + 1] if l + 1 < len(self.blocks) else None
+            # x_{l+1} and, for the next block, its router logits, from one read of x_l and y_l
+            x, logits = self.residual_router(x, y, nxt.w_r if nxt else None,
+                                             nxt.b_r if nxt else None)
         return x, saved
 
     def backward(self, dy: torch.Tensor, saved: list, tap: Callable | None = None):
@@ -123,15 +116,14 @@ class MoeStack:
         g = dy
         for l in reversed(range(len(self.blocks))):
             b = self.blocks[l]
-            x = saved[l]
-            logits = router_logits(x, b.w_r, b.b_r)
+            x, logits = saved[l]
             self.block_forward(l, x, logits)  # recompute: refills the block's saved state
             out = self.block_backward(l, g)
             dx_moe, d_logits = out[0], out[1]
             if tap is not None:
                 tap(l, {"g": g, "dx": dx_moe, "d_logits": d_logits,
                         "d_w": out[2] if len(out) > 2 else None})
-            g = grad_chain(g, dx_moe, d_logits, b.w_r)
+            g = self.grad_chain(g, dx_moe, d_logits, b.w_r)
         return g
 
 

@@ -205,3 +205,33 @@ def test_binding_without_the_library_fails_loudly(tmp_path):
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
                        cwd=str(tmp_path))
     assert r.returncode == 3 and "IMPORT_ERROR" in r.stdout, r.stdout + r.stderr
+
+
+def test_residual_entry_points_validate_before_the_device(L):
+    """Bad shapes, missing operands, misalignment and an output overlapping an input are
+    INVALID_ARG without any device call; a valid call reaches the device check (no GPU here)."""
+    a = ctypes.c_void_p(1 << 20)          # 16-byte aligned addresses, never dereferenced
+    b = ctypes.c_void_p((1 << 20) + (1 << 16))
+    c = ctypes.c_void_p((1 << 20) + (2 << 16))
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    rr = L.lib.mxfp4_moe_residual_router
+    bad = [
+        (4, 48, 8, a, b, a, None, c, None),     # H not a multiple of 32
+        (4, 64, 0, a, b, a, None, c, None),     # E = 0
+        (4, 64, 300, a, b, a, None, c, None),   # E > 256
+        (4, 64, 8, None, b, a, None, c, None),  # no x
+        (4, 64, 8, a, None, None, None, None, None),  # neither a residual nor logits
+        (4, 64, 8, a, b, a, None, None, None),  # y without x_out
+        (4, 64, 8, a, None, a, None, c, a),     # x_out without y
+        (4, 64, 8, a, b, None, None, c, a),     # logits without w_r
+        (4, 64, 8, odd, b, a, None, c, None),   # misaligned x
+        (4, 64, 8, a, b, a, None, a, None),     # x_out overlaps x
+    ]
+    for args in bad:
+        assert rr(*args, None) == L.ERR_INVALID_ARG, args
+    assert rr(4, 64, 8, a, b, a, None, c, a, None) in (L.ERR_UNSUPPORTED_DEVICE, L.ERR_CUDA)
+    gc = L.lib.mxfp4_moe_grad_chain
+    for args in [(4, 48, 8, a, b, c, a, a), (4, 64, 0, a, b, c, a, a), (4, 64, 8, None, b, c, a, a),
+                 (4, 64, 8, a, b, None, a, a), (4, 64, 8, a, b, c, odd, a)]:
+        assert gc(*args, None) == L.ERR_INVALID_ARG, args
+    assert gc(4, 64, 8, a, b, c, a, a, None) in (L.ERR_UNSUPPORTED_DEVICE, L.ERR_CUDA)

@@ -8,6 +8,10 @@ through the stack harness's forward and its recompute-per-block backward:
 * the full stack (24 gpt-oss-20b blocks, T=32768) on 16 sampled tokens, since each token's
   path through the stack is independent of the other tokens.
 
+Between the blocks, the library's two caller-side kernels are checked on the same tokens:
+x_{l+1} = bf16(x_l + y_l) bit for bit, the logits of every block against x_l W_r + b_r in
+fp64, and each upstream gradient g_l against g_{l+1} + dX_l + d_logits_l W_r^T in fp64.
+
 The stack output is not compared end to end with an fp64 chain: the caller rounds the
 residual stream to bf16 after every block, and a difference at that rounding flips top-k
 and clamp decisions downstream (an fp64 emulation of the bf16 stream alone drifts to cosine
@@ -27,6 +31,7 @@ from mxfp4_quantized_moe_b200 import inputs, stack
 
 import oracle_pool
 from test_gpu_parity import _ws_offsets, assert_close, assert_d_logits_close
+from test_gpu_residual import _check_logits
 
 pytestmark = pytest.mark.gpu
 
@@ -60,6 +65,9 @@ def _run_blockwise(wl, seed, sel, workers=1):
     out, saved = st.forward(x, tap=tap_f)
     g0 = st.backward(dy, saved, tap=tap_b)
     torch.cuda.synchronize()
+    w_r = [b.w_r.cpu() for b in blocks]
+    b_r = [b.b_r.cpu() for b in blocks]
+    g0_sel = g0[selc].cpu()
     rc, where = moe.device_check(st.ws)
     assert rc == 0, f"device error {rc} at {where:#x}"
     assert torch.isfinite(out.float()).all() and torch.isfinite(g0.float()).all()
@@ -76,6 +84,23 @@ def _run_blockwise(wl, seed, sel, workers=1):
             refs = list(ex.map(oracle_pool.block, jobs))
     else:
         refs = [oracle_pool.block(j) for j in jobs]
+    # the caller-side kernels between the blocks
+    for l in range(wl.layers):
+        if l == 0:
+            _check_logits(fw[0]["logits"], fw[0]["x"], w_r[0], b_r[0])
+        if l + 1 < wl.layers:
+            ref_x = (fw[l]["x"].float() + fw[l]["y"].float()).to(torch.bfloat16)
+            assert torch.equal(fw[l + 1]["x"], ref_x), f"x[{l + 1}] is not bf16(x + y)"
+            _check_logits(fw[l + 1]["logits"], fw[l + 1]["x"], w_r[l + 1], b_r[l + 1])
+        # g_l, the upstream gradient of block l - 1 (of the stack input for l = 0)
+        g_l = bw[l - 1]["g"] if l > 0 else g0_sel
+        parts = [bw[l]["g"].double().numpy(), bw[l]["dx"].double().numpy(),
+                 bw[l]["d_logits"].double().numpy() @ w_r[l].double().numpy().T]
+        ref = sum(parts)
+        scale = sum(np.abs(p) for p in parts[:2]) + \
+            np.abs(bw[l]["d_logits"].double().numpy()) @ np.abs(w_r[l].double().numpy()).T
+        err = np.abs(g_l.double().numpy() - ref)
+        assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-5 * scale + 1e-30), f"g[{l}]"
     for l, (out, dX, d_w, d_logits, w, y_abs) in enumerate(refs):
         assert_close(_np(fw[l]["y"]), out, f"y[{l}]")
         assert_close(_np(bw[l]["dx"]), dX, f"dx[{l}]")

@@ -92,7 +92,16 @@ def test_harness_chaining_matches_oracle_stack():
 
     blocks = [StackBlock(None, None, torch.from_numpy(ly["w_r"]), torch.from_numpy(ly["b_r"]))
               for ly in layers]
-    st = MoeStack(None, blocks, block_forward=block_forward, block_backward=block_backward)
+    def residual_router(xt, y, w_r, b_r):  # the caller-side steps by definition, in fp64
+        x_next = None if y is None else xt + y
+        xs = xt if y is None else x_next
+        return x_next, (None if w_r is None else xs @ w_r + b_r)
+
+    def grad_chain(g, dx, d_logits, w_r):
+        return g + dx + d_logits @ w_r.T
+
+    st = MoeStack(None, blocks, block_forward=block_forward, block_backward=block_backward,
+                  residual_router=residual_router, grad_chain=grad_chain)
     xt = torch.from_numpy(x.copy())
     out, saved = st.forward(xt)
     calls_fwd = list(calls)
@@ -106,4 +115,5 @@ def test_harness_chaining_matches_oracle_stack():
     # its backward, from the last block down
     assert calls_fwd == [("f", l) for l in range(L)]
     assert calls[L:] == [c for l in reversed(range(L)) for c in (("f", l), ("b", l))]
-    assert len(saved) == L and all(s.shape == (T, H) for s in saved)
+    assert len(saved) == L and all(s[0].shape == (T, H) and s[1].shape == (T, E)
+                                   for s in saved)
