@@ -273,7 +273,8 @@ MXFP4_MOE_API int mxfp4_moe_residual_router(int32_t T, int32_t H, int32_t E, con
 /* The residual stream's gradient through one stacked block, in one kernel (source as for
  * mxfp4_moe_residual_router):
  *   g_out[t][h] = bf16(g[t][h] + dx[t][h] + sum_e d_logits[t][e] * w_r[h][e])
- * in fp32 (the sum over e in ascending order, then g + dx + that sum), rounded once.
+ * in fp32 (fused multiply-adds over e in ascending order, then g + dx + that sum), rounded
+ * once.
  *   g, dx, g_out  bf16 [T][H] DEVICE, 16-byte aligned; g_out may be g itself
  *   d_logits      fp32 [T][E] DEVICE (mxfp4_moe_backward_input's router gradient)
  *   w_r           bf16 [H][E] DEVICE, 16-byte aligned

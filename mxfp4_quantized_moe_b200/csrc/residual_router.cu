@@ -178,104 +178,100 @@ __global__ void __launch_bounds__(kThreads, 4) residual_router_kernel(
 }
 
 // ---- grad_chain ------------------------------------------------------------------------
-// g_out = bf16(g + dx + d_logits W_r^T): a GEMM over the experts (K = E, up to 256) with the
-// tokens as M and the features as N.  d_logits is fp32: each value splits exactly into three
-// bf16 parts (hi = bf16(v), mid = bf16(v - hi), lo = v - hi - mid; 8 significant bits each,
-// 24 in all), and the three products with the bf16 W_r accumulate in fp32, so the sum keeps
-// fp32 operands.  The CTA's d_logits rows stay in shared memory; each chunk of 64 features
-// stages its rows of W_r (zero-padded to whole k-steps), whose B fragments are plain 32-bit
-// loads ([h][e] rows are k-contiguous).
-MOE_DEV void split3(float v, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
-  const uint16_t h = f_to_bf16(v);
-  const float r1 = v - bf16_to_f(h);
-  const uint16_t m = f_to_bf16(r1);
-  const uint16_t l = f_to_bf16(r1 - bf16_to_f(m));
-  hi = h; mid = m; lo = l;
-}
+// g_out = bf16(g + dx + d_logits W_r^T) in fp32 on the CUDA cores: a CTA takes 64 tokens and
+// walks H in chunks of 64 features; thread (tg, hg) forms the 4 x 8 block of tokens 4 tg..+3
+// and features 8 hg..+7 of the chunk, summing the experts in ascending order with fp32 FMAs
+// from two transposed shared-memory tiles (d_logits [e][token] for the CTA, W_r [e][h] for
+// the chunk; per expert one 16-byte load of d_logits and two of W_r feed 32 FMAs), then adds
+// g and dx (requested before the FMAs) and rounds once.
+constexpr int kGCTok = 64, kGCH = 64;
 
 __global__ void __launch_bounds__(kThreads) grad_chain_kernel(
     int T, int H, int E, const uint16_t* __restrict__ g, const uint16_t* __restrict__ dx,
     const float* __restrict__ d_logits, const uint16_t* __restrict__ w_r,
-    uint16_t* __restrict__ g_out, int ek, int dpitch, int wpitch) {
-  // ek: E rounded up to a whole k-step (16); dpitch: fp32 row pitch of d_logits (ek + 8, so
-  // that the 64-bit fragment loads of a half-warp hit distinct banks); wpitch: bf16 row pitch
-  // of the W_r chunk (ek + 8: 4 (2 ek/16 + 1) words, conflict-free 32-bit fragment loads)
+    uint16_t* __restrict__ g_out) {
   extern __shared__ __align__(16) float s_dyn[];
-  float* s_dl = s_dyn;                                               // [64][dpitch]
-  uint16_t* s_w = reinterpret_cast<uint16_t*>(s_dl + kTok * dpitch);  // [64][wpitch]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gr = lane >> 2, c = lane & 3;
-  const int t0 = blockIdx.x * kTok;
-  for (int i = threadIdx.x; i < kTok * ek; i += kThreads) {
-    const int r = i / ek, e = i % ek;
+  float* s_dl = s_dyn;                // [E][kGCTok]
+  float* s_w = s_dyn + E * kGCTok;    // [E][kGCH]
+  const int t0 = blockIdx.x * kGCTok;
+  const int tg = threadIdx.x >> 3, hg = threadIdx.x & 7;  // 16 token groups x 8 feature groups
+  for (int i = threadIdx.x; i < kGCTok * E; i += kThreads) {  // consecutive threads: tokens
+    const int r = i % kGCTok, e = i / kGCTok;
     const int t = t0 + r;
-    s_dl[r * dpitch + e] = (t < T && e < E) ? __ldg(d_logits + (size_t)t * E + e) : 0.f;
+    s_dl[e * kGCTok + r] = (t < T) ? __ldg(d_logits + (size_t)t * E + e) : 0.f;
   }
-  const int nchunk = (H + kChunk - 1) / kChunk;
+  const int nchunk = (H + kGCH - 1) / kGCH;
   for (int kc = 0; kc < nchunk; ++kc) {
-    const int h0 = kc * kChunk;
-    __syncthreads();  // d_logits staged / the previous chunk's W_r rows read
-    if ((E & 7) == 0) {  // rows of W_r in whole 16-byte vectors (wpitch keeps rows aligned)
-      const int nv = ek / 8;
-      for (int i = threadIdx.x; i < kChunk * nv; i += kThreads) {
-        const int hh = i / nv, cv = i % nv;
-        const int h = h0 + hh, e = 8 * cv;
+    const int h0 = kc * kGCH;
+    __syncthreads();  // d_logits staged / the previous chunk's W_r tile read
+    if ((E & 7) == 0) {  // 16-byte vectors of 8 experts (w_r is 16-byte aligned)
+      for (int i = threadIdx.x; i < kGCH * (E / 8); i += kThreads) {  // consecutive: features
+        const int hh = i % kGCH, e = 8 * (i / kGCH);
+        const int h = h0 + hh;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (h < H && e < E) v = __ldg(reinterpret_cast<const uint4*>(w_r + (size_t)h * E + e));
-        *reinterpret_cast<uint4*>(s_w + hh * wpitch + e) = v;
+        if (h < H) v = __ldg(reinterpret_cast<const uint4*>(w_r + (size_t)h * E + e));
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          s_w[(e + 2 * q) * kGCH + hh] = bf16_lo(vw[q]);
+          s_w[(e + 2 * q + 1) * kGCH + hh] = bf16_hi(vw[q]);
+        }
       }
     } else {
-      for (int i = threadIdx.x; i < kChunk * ek; i += kThreads) {
-        const int hh = i / ek, e = i % ek;
+      for (int i = threadIdx.x; i < kGCH * E; i += kThreads) {  // consecutive threads: features
+        const int hh = i % kGCH, e = i / kGCH;
         const int h = h0 + hh;
-        s_w[hh * wpitch + e] = (h < H && e < E) ? __ldg(w_r + (size_t)h * E + e) : (uint16_t)0;
+        s_w[e * kGCH + hh] = (h < H) ? bf16_to_f(__ldg(w_r + (size_t)h * E + e)) : 0.f;
       }
     }
     __syncthreads();
-    float acc[kChunk / 8][4];
+    // this thread's g and dx vectors of the chunk, requested before the FMAs so that their
+    // latency overlaps them (H % 32 == 0: the 8 features are all in range or all out)
+    const int h = h0 + 8 * hg;
+    uint4 gv[4], dv4[4];
 #pragma unroll
-    for (int n = 0; n < kChunk / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    const float* da = s_dl + (16 * warp) * dpitch;
-    for (int kk = 0; kk < ek; kk += 16) {
-      // A fragments (rows gr, gr+8; experts kk + 2c (+1), kk + 8 + 2c (+1)) in three parts
-      uint32_t ah[4], am[4], al[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int row = gr + 8 * (q & 1), col = kk + 2 * c + 8 * (q >> 1);
-        const float2 v = *reinterpret_cast<const float2*>(da + row * dpitch + col);
-        uint32_t h0_, m0_, l0_, h1_, m1_, l1_;
-        split3(v.x, h0_, m0_, l0_);
-        split3(v.y, h1_, m1_, l1_);
-        ah[q] = h0_ | (h1_ << 16);
-        am[q] = m0_ | (m1_ << 16);
-        al[q] = l0_ | (l1_ << 16);
-      }
-#pragma unroll
-      for (int n = 0; n < kChunk / 8; ++n) {
-        const uint16_t* wb = s_w + (8 * n + gr) * wpitch + kk + 2 * c;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wb);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wb + 8);
-        mma_16816(acc[n], al, b0, b1);  // smallest part first
-        mma_16816(acc[n], am, b0, b1);
-        mma_16816(acc[n], ah, b0, b1);
+    for (int r = 0; r < 4; ++r) {
+      const int t = t0 + 4 * tg + r;
+      gv[r] = dv4[r] = make_uint4(0u, 0u, 0u, 0u);
+      if (t < T && h < H) {
+        const size_t at = ((size_t)t * H + h) / 8;
+        gv[r] = reinterpret_cast<const uint4*>(g)[at];
+        dv4[r] = __ldg(reinterpret_cast<const uint4*>(dx) + at);
       }
     }
-    // g_out for tokens 16 warp + gr (+8), features h0 + 8n + 2c (+1): two bf16 per word
+    float acc[4][8];
 #pragma unroll
-    for (int n = 0; n < kChunk / 8; ++n) {
+    for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int t = t0 + 16 * warp + gr + 8 * half;
-        const int h = h0 + 8 * n + 2 * c;
-        if (t < T && h < H) {
-          const size_t at = ((size_t)t * H + h) / 2;
-          const uint32_t gv = reinterpret_cast<const uint32_t*>(g)[at];
-          const uint32_t dv = __ldg(reinterpret_cast<const uint32_t*>(dx) + at);
-          const float s0 = bf16_lo(gv) + bf16_lo(dv) + acc[n][2 * half];
-          const float s1 = bf16_hi(gv) + bf16_hi(dv) + acc[n][2 * half + 1];
-          reinterpret_cast<uint32_t*>(g_out)[at] = pack_bf16x2(s0, s1);
-        }
-      }
+      for (int j = 0; j < 8; ++j) acc[r][j] = 0.f;
+    const float* dl = s_dl + 4 * tg;
+    const float* wv = s_w + 8 * hg;
+#pragma unroll 4
+    for (int e = 0; e < E; ++e) {
+      const float4 d = *reinterpret_cast<const float4*>(dl + e * kGCTok);
+      const float4 w0 = *reinterpret_cast<const float4*>(wv + e * kGCH);
+      const float4 w1 = *reinterpret_cast<const float4*>(wv + e * kGCH + 4);
+      const float dv[4] = {d.x, d.y, d.z, d.w};
+      const float ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[r][j] = fmaf(dv[r], ww[j], acc[r][j]);
+    }
+    if (h >= H) continue;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int t = t0 + 4 * tg + r;
+      if (t >= T) continue;
+      const size_t at = ((size_t)t * H + h) / 8;
+      const uint32_t gw[4] = {gv[r].x, gv[r].y, gv[r].z, gv[r].w};
+      const uint32_t dw[4] = {dv4[r].x, dv4[r].y, dv4[r].z, dv4[r].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o[q] = pack_bf16x2(bf16_lo(gw[q]) + bf16_lo(dw[q]) + acc[r][2 * q],
+                           bf16_hi(gw[q]) + bf16_hi(dw[q]) + acc[r][2 * q + 1]);
+      reinterpret_cast<uint4*>(g_out)[at] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 }
@@ -295,22 +291,18 @@ cudaError_t launch_residual_router(int T, int H, int E, const uint16_t* x, const
   return cudaGetLastError();
 }
 
-size_t grad_chain_smem_bytes(int E) {
-  const int ek = (E + 15) / 16 * 16;
-  return (size_t)kTok * (ek + 8) * 4 + (size_t)kChunk * (ek + 8) * 2;
-}
+size_t grad_chain_smem_bytes(int E) { return (size_t)E * (kGCTok + kGCH) * 4; }
 
 cudaError_t launch_grad_chain(int T, int H, int E, const uint16_t* g, const uint16_t* dx,
                               const float* d_logits, const uint16_t* w_r, uint16_t* g_out,
                               cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const int ek = (E + 15) / 16 * 16;
   const size_t smem = grad_chain_smem_bytes(E);
   cudaError_t e = cudaFuncSetAttribute(grad_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  grad_chain_kernel<<<(T + kTok - 1) / kTok, kThreads, smem, st>>>(T, H, E, g, dx, d_logits, w_r,
-                                                                   g_out, ek, ek + 8, ek + 8);
+  grad_chain_kernel<<<(T + kGCTok - 1) / kGCTok, kThreads, smem, st>>>(T, H, E, g, dx, d_logits,
+                                                                       w_r, g_out);
   return cudaGetLastError();
 }
 
