@@ -15,8 +15,7 @@ namespace moe {
 
 namespace {
 
-// Both kernels take 64 tokens per CTA (4 warps x 16 rows of an m16n8k16 bf16 mma.sync tile,
-// fp32 accumulation) through H in chunks of 64.
+// Both kernels take 64 tokens per CTA through H in chunks of 64 features.
 constexpr int kTok = 64;
 constexpr int kChunk = 64;
 constexpr int kThreads = 128;
@@ -41,6 +40,7 @@ MOE_DEV uint32_t add_bf16x2_rn(uint32_t a, uint32_t b) {  // fp32 sums rounded o
 }
 
 // ---- residual_router ------------------------------------------------------------------
+// 4 warps x 16 tokens, each warp's logits on m16n8k16 bf16 mma.sync tiles (fp32 accumulation).
 // Per chunk: x_out = x + y for the CTA's 64 tokens (16-byte vectors: x_out to memory and to
 // shared memory as the A operand) and the chunk of W_r as stored ([h][e], 16-byte vectors),
 // whose B fragments ldmatrix.trans reads; the next chunk's loads are in flight while the MMAs
@@ -291,7 +291,7 @@ cudaError_t launch_residual_router(int T, int H, int E, const uint16_t* x, const
   return cudaGetLastError();
 }
 
-size_t grad_chain_smem_bytes(int E) { return (size_t)E * (kGCTok + kGCH) * 4; }
+static size_t grad_chain_smem_bytes(int E) { return (size_t)E * (kGCTok + kGCH) * 4; }
 
 cudaError_t launch_grad_chain(int T, int H, int E, const uint16_t* g, const uint16_t* dx,
                               const float* d_logits, const uint16_t* w_r, uint16_t* g_out,
