@@ -270,8 +270,9 @@ MXFP4_MOE_API int mxfp4_moe_residual_router(int32_t T, int32_t H, int32_t E, con
                                             const uint16_t* b_r, uint16_t* x_out,
                                             float* logits, void* stream);
 
-/* The residual stream's gradient through one stacked block, in one kernel (source as for
- * mxfp4_moe_residual_router):
+/* The residual stream's gradient through one stacked block, in one kernel.  Source: "Add
+ * MXFP4 training support via a dequantize-on-the-fly fallback", section "What this does"
+ * (the backward of gradient-checkpointed decoder layers); the fusion has no counterpart there.
  *   g_out[t][h] = bf16(g[t][h] + dx[t][h] + sum_e d_logits[t][e] * w_r[h][e])
  * in fp32 (fused multiply-adds over e in ascending order, then g + dx + that sum), rounded
  * once.
