@@ -633,11 +633,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j)
           dnext[j] = __ldg(p.dgu + (size_t)min(tl.row0 + j, p.A - 1) * N + f);
       }
-      if (!mbar_wait_sleep(smem_u32(&bar->acc_full[acc]), (lt / kAccBufs) & 1, err, 0x500, s_abort, 256)) break;
-      tc_fence_after();
+      // the bias (gate_up, down) and dact's routing weights of the tile's rows (lane l holds
+      // row 32 c + l of chunk c) are requested before the accumulator is ready, so that no
+      // global load sits between the accumulator and its release
       float bias_f = 0.f;
       if ((EPI == kEpiGateUp || EPI == kEpiDown) && active)
         bias_f = bf16_to_f(p.bias[(size_t)tl.e * N + f]);
+      float wrow[kBN / 32];
+      if (EPI == kEpiDact) {
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c)
+          wrow[c] = (32 * c + lane < tl.n_valid) ? p.w_row[tl.row0 + 32 * c + lane] : 0.f;
+      }
+      if (!mbar_wait_sleep(smem_u32(&bar->acc_full[acc]), (lt / kAccBufs) & 1, err, 0x500, s_abort, 256)) break;
+      tc_fence_after();
       const uint32_t acc_tmem = tmem + ((uint32_t)(32 * q) << 16) + acc * kAccCols;
       const bool odd = (lane & 1) != 0;
       if (EPI != kEpiDact) {
@@ -768,9 +777,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // dact keeps the fp32 accumulator through its multiply: chunk by chunk, then release
+        // one chunk per pass (rolled, as for the GLU): the routing weights move down one slot
+        // per pass, so the current chunk's are always in wrow[0]
+#pragma unroll 1
         for (int c0 = 0; c0 < tl.n_valid; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(acc_tmem + c0, r);
+          const float my_w = wrow[0];
+#pragma unroll
+          for (int cc = 0; cc + 1 < kBN / 32; ++cc) wrow[cc] = wrow[cc + 1];
           tmem_wait_ld();
           if (!active) continue;
           const int ncol = min(32, tl.n_valid - c0);
@@ -779,7 +794,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           // from the factors the forward saved.
           const int I = N;
           uint32_t* dh = reinterpret_cast<uint32_t*>(p.out0);
-          const float my_w = (lane < ncol) ? p.w_row[rbase + lane] : 0.f;
           uint32_t dcur[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) dcur[j] = dnext[j];
