@@ -61,10 +61,10 @@ def peaks():
 # only while the kernel's sources hash to `sources`: after any change it reads as null.
 NCU_TRAFFIC = {
     # profiles/launch_list_gpt-oss-20b-moe-T8192.md (one launch of each after three warm-up steps)
-    ("gemm_gate_up_glu", "gpt-oss-20b-moe-T8192"): {"bytes": 472046848 + 524553216, "sources": "308883011b4735fd"},
-    ("gemm_down", "gpt-oss-20b-moe-T8192"): {"bytes": 330158848 + 157707776, "sources": "308883011b4735fd"},
-    ("gemm_dact_glu_bwd", "gpt-oss-20b-moe-T8192"): {"bytes": 707796224 + 344864256, "sources": "308883011b4735fd"},
-    ("gemm_dx", "gpt-oss-20b-moe-T8192"): {"bytes": 673688576 + 170546688, "sources": "308883011b4735fd"},
+    ("gemm_gate_up_glu", "gpt-oss-20b-moe-T8192"): {"bytes": 471644928 + 525486080, "sources": "985c6c401244b781"},
+    ("gemm_down", "gpt-oss-20b-moe-T8192"): {"bytes": 330095616 + 157613056, "sources": "985c6c401244b781"},
+    ("gemm_dact_glu_bwd", "gpt-oss-20b-moe-T8192"): {"bytes": 710861824 + 343664128, "sources": "985c6c401244b781"},
+    ("gemm_dx", "gpt-oss-20b-moe-T8192"): {"bytes": 669618944 + 170102016, "sources": "985c6c401244b781"},
 }
 KERNEL_SOURCES = ("mxfp4_quantized_moe_b200/csrc/grouped_gemm.cu",
                   "mxfp4_quantized_moe_b200/csrc/common.cuh",
